@@ -1,0 +1,293 @@
+"""Plain, slow CPU oracle of the Self-Indexing KVCache decode hot path.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import or run anything in
+this package.  The product (the CUDA library and its Python binding) never
+imports it and shares no code with it; the two meet only at the seeded inputs
+of ``sikv_inputs``.
+
+Source of every step: "Self-Indexing KVCache: Predicting Sparse Attention from
+Compressed Keys" (summary page at gist.science, paper 2603.14224), cited below
+as [SIKV §x] for section x of its technical summary:
+
+* §2.1.1  sign-based 1-bit vector quantization: entropy-aware (channel mean)
+          normalization, 4-dim sub-vectors mapped by their sign pattern to one
+          of 16 clusters, one-pass (non-iterative) clustering into a codebook;
+          the same code serves reconstruction and top-k retrieval;
+* §2.1.2  compressed-domain top-k retrieval by LUT-GEMV: the query is split
+          like the key, dotted with the 16 centroids of each subspace to form a
+          lookup table, and a key's score is the sum of the table entries its
+          codes index;
+* §2.1.3  token-wise format and 64 full-precision sink tokens kept from prefill;
+* §2.1.4  dequantization fused with the sparse attention pass.
+
+Where the page is silent the plainest reading is taken; each one is tagged
+[R#] and listed in the design notes of the repository:
+
+R1  the mean is per (sequence, KV head, channel) over the prefill keys;
+R2  sinks are tokens 0..S-1; they are excluded from the mean, the codebook and
+    scoring, and are always attended with their stored K and V;
+R3  the mean is the exact mean rounded once to fp32, and that fp32 value is
+    what the sign decision compares against;
+R4  bit i of a sub-vector's code is [k_{4s+i} >= mu_{4s+i}] (ties give 1),
+    LSB first;
+R5  sub-vectors are the contiguous dimensions [4s, 4s+4);
+R6  two codes per byte, even subspace in the low nibble, one 16-byte row per
+    token;
+R7  a centroid is the arithmetic mean of the normalized sub-vectors (k - mu)
+    of its cluster;
+R8  an empty cluster has centroid 0;
+R9  the query heads of a GQA group share one selection, scored with the sum
+    of their queries;
+R10 softmax scale 1/sqrt(D);
+R11 k counts non-sink tokens only;
+R12 top-k ties go to the lower token index;
+R13 the selected set is returned in ascending token order;
+R14 a selected key is reconstructed as mu + c[s][code_s].
+"""
+
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+SUB_DIM = 4          # [SIKV §2.1.1]: 4-dimensional sub-vectors
+NUM_CLUSTERS = 16    # [SIKV §2.1.1]: sign pattern of 4 dims -> one of 16 clusters
+DEFAULT_SINKS = 64   # [SIKV §2.1.3]: 64 full-precision sink tokens
+
+
+# ----------------------------------------------------------------------------
+# exact arithmetic helpers
+# ----------------------------------------------------------------------------
+
+def exact_sum(values) -> Fraction:
+    """Exact sum of floats.
+
+    ``math.fsum`` returns the correctly rounded sum; appending its negation and
+    summing again yields the correctly rounded remainder, which is 0 exactly
+    when nothing is left.  The remainder shrinks by at least 2**52 per round.
+    """
+    terms = [float(v) for v in values]
+    total = Fraction(0)
+    while True:
+        s = math.fsum(terms)
+        if s == 0.0:
+            return total
+        total += Fraction(s)
+        terms.append(-s)
+
+
+def round_to_f32(x: Fraction) -> np.float32:
+    """Round an exact rational to the nearest fp32, ties to even."""
+    c = np.float32(float(x))
+    cands = [np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))]
+    best, best_d = None, None
+    for cand in cands:
+        if not np.isfinite(cand):
+            continue
+        d = abs(Fraction(float(cand)) - x)
+        if best is None or d < best_d or (d == best_d and int(np.float32(cand).view(np.uint32)) % 2 == 0):
+            best, best_d = np.float32(cand), d
+    return best
+
+
+# ----------------------------------------------------------------------------
+# prefill: encode the key cache  [SIKV §2.1.1, §2.1.3]
+# ----------------------------------------------------------------------------
+
+def channel_mean(K: np.ndarray, num_sinks: int = DEFAULT_SINKS) -> np.ndarray:
+    """Entropy-aware normalization mean [SIKV §2.1.1] (R1, R2, R3).
+
+    mu[c] = (1/n) * sum_{t=S}^{N-1} K[t, c], computed exactly and rounded once
+    to fp32.  With no non-sink token (N <= S) the mean is 0.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    n_tok, d = K.shape
+    rows = K[num_sinks:]
+    n = rows.shape[0]
+    mu = np.zeros(d, dtype=np.float32)
+    if n == 0:
+        return mu
+    for c in range(d):
+        mu[c] = round_to_f32(exact_sum(rows[:, c].tolist()) / n)
+    return mu
+
+
+def sign_codes(K: np.ndarray, mu: np.ndarray) -> np.ndarray:
+    """Sign-pattern code of every 4-dim sub-vector [SIKV §2.1.1] (R4, R5).
+
+    code[t, s] = sum_i [K[t, 4s+i] >= mu[4s+i]] * 2**i, one nibble per
+    (token, subspace).  All tokens get a code, sinks included; sinks' codes are
+    never used.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    mu = np.asarray(mu, dtype=np.float32).astype(np.float64)
+    n_tok, d = K.shape
+    p = d // SUB_DIM
+    bits = (K >= mu[None, :]).astype(np.uint8).reshape(n_tok, p, SUB_DIM)
+    code = np.zeros((n_tok, p), dtype=np.uint8)
+    for i in range(SUB_DIM):
+        code |= bits[:, :, i] << i
+    return code
+
+
+def pack_codes(code: np.ndarray) -> np.ndarray:
+    """Token-wise packed layout [SIKV §2.1.3] (R6): byte m = code[2m] | code[2m+1] << 4."""
+    code = np.asarray(code, dtype=np.uint8)
+    if code.shape[1] % 2:
+        raise ValueError("packing needs an even number of subspaces (D a multiple of 8)")
+    return (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack_codes`."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    n, m = packed.shape
+    code = np.zeros((n, 2 * m), dtype=np.uint8)
+    code[:, 0::2] = packed & 0x0F
+    code[:, 1::2] = packed >> 4
+    return code
+
+
+def codebook(K: np.ndarray, mu: np.ndarray, code: np.ndarray, num_sinks: int = DEFAULT_SINKS):
+    """One-pass sign-pattern clustering [SIKV §2.1.1] (R2, R7, R8).
+
+    c[s][j] = mean over non-sink tokens t with code[t, s] == j of the
+    normalized sub-vector K[t, 4s:4s+4] - mu[4s:4s+4]; 0 for an empty cluster.
+    Returns (centroids float64 [P][16][4], counts int64 [P][16]).
+    """
+    K = np.asarray(K, dtype=np.float64)
+    mu64 = np.asarray(mu, dtype=np.float32).astype(np.float64)
+    n_tok, d = K.shape
+    p = d // SUB_DIM
+    cent = np.zeros((p, NUM_CLUSTERS, SUB_DIM))
+    counts = np.zeros((p, NUM_CLUSTERS), dtype=np.int64)
+    x = K[num_sinks:] - mu64[None, :]
+    cs = code[num_sinks:]
+    for s in range(p):
+        xs = x[:, SUB_DIM * s:SUB_DIM * (s + 1)]
+        for j in range(NUM_CLUSTERS):
+            members = cs[:, s] == j
+            cnt = int(members.sum())
+            counts[s, j] = cnt
+            if cnt:
+                cent[s, j] = xs[members].mean(axis=0)
+    return cent, counts
+
+
+def encode_keys(K: np.ndarray, num_sinks: int = DEFAULT_SINKS):
+    """Whole prefill encoder for one (sequence, KV head).
+
+    Returns (mu fp32 [D], codes uint8 [N][P] one nibble per entry, centroids
+    f64 [P][16][4], counts [P][16]); :func:`pack_codes` gives the stored rows.
+    """
+    mu = channel_mean(K, num_sinks)
+    code = sign_codes(K, mu)
+    cent, counts = codebook(K, mu, code, num_sinks)
+    return mu, code, cent, counts
+
+
+def reconstruct_keys(mu: np.ndarray, centroids: np.ndarray, code: np.ndarray) -> np.ndarray:
+    """Dequantized keys k_hat[t] = mu + c[s][code[t, s]] per subspace (R14)."""
+    mu64 = np.asarray(mu, dtype=np.float32).astype(np.float64)
+    n_tok, p = code.shape
+    k_hat = np.empty((n_tok, p * SUB_DIM))
+    for s in range(p):
+        k_hat[:, SUB_DIM * s:SUB_DIM * (s + 1)] = centroids[s][code[:, s]]
+    return k_hat + mu64[None, :]
+
+
+# ----------------------------------------------------------------------------
+# decode: compressed-domain scoring  [SIKV §2.1.2]
+# ----------------------------------------------------------------------------
+
+def group_query(q_group: np.ndarray) -> np.ndarray:
+    """Summed query of a GQA group (R9): q_bar = sum_h q_h."""
+    return np.asarray(q_group, dtype=np.float64).sum(axis=0)
+
+
+def lut(q_bar: np.ndarray, centroids: np.ndarray) -> np.ndarray:
+    """Lookup table [SIKV §2.1.2]: LUT[s][j] = q_bar[4s:4s+4] . c[s][j]."""
+    p = centroids.shape[0]
+    qs = np.asarray(q_bar, dtype=np.float64).reshape(p, SUB_DIM)
+    return np.einsum("si,sji->sj", qs, centroids)
+
+
+def scores(q_group: np.ndarray, mu: np.ndarray, centroids: np.ndarray, code: np.ndarray,
+           num_sinks: int = DEFAULT_SINKS):
+    """LUT-GEMV scores of every token [SIKV §2.1.2] (R2, R9).
+
+    score[t] = sum_s LUT[s][code[t, s]] + q_bar . mu for t >= S, -inf for sinks.
+    Also returns the condition scale sum_s |LUT[s][code[t, s]]| + |q_bar . mu|
+    that bounds the rounding error of any evaluation order of that sum.
+    """
+    q_bar = group_query(q_group)
+    table = lut(q_bar, centroids)
+    n_tok, p = code.shape
+    picked = table[np.arange(p)[None, :], code.astype(np.int64)]        # [N][P]
+    qmu = float(np.dot(q_bar, np.asarray(mu, dtype=np.float32).astype(np.float64)))
+    sc = picked.sum(axis=1) + qmu
+    scale = np.abs(picked).sum(axis=1) + abs(qmu)
+    sc[:min(num_sinks, n_tok)] = -np.inf
+    return sc, scale
+
+
+def topk(score: np.ndarray, k: int, num_sinks: int = DEFAULT_SINKS) -> np.ndarray:
+    """Top-k over the non-sink tokens (R11, R12, R13).
+
+    Orders tokens t in [S, N) by (-score[t], t) and keeps the first k; returns
+    them in ascending token order.  -0.0 and +0.0 compare equal.
+    """
+    score = np.asarray(score, dtype=np.float64)
+    n_tok = score.shape[0]
+    cand = np.arange(num_sinks, n_tok)
+    if k < 0 or k > cand.size:
+        raise ValueError(f"k={k} outside [0, {cand.size}]")
+    order = np.lexsort((cand, -score[cand]))
+    return np.sort(cand[order[:k]]).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------
+# decode: sparse attention over sinks + selected tokens  [SIKV §2.1.3, §2.1.4]
+# ----------------------------------------------------------------------------
+
+def sparse_attention(q_group: np.ndarray, K: np.ndarray, V: np.ndarray, mu: np.ndarray,
+                     centroids: np.ndarray, code: np.ndarray, idx: np.ndarray,
+                     num_sinks: int = DEFAULT_SINKS, scale: float | None = None) -> np.ndarray:
+    """Attention of each query head over T = {0..S-1} (full precision) and idx.
+
+    logit_t = scale * q_h . K[t] for a sink, scale * q_h . (mu + c[code_t]) for
+    a selected token (R14); out_h = sum_t softmax(logit)_t V[t] (R10).
+    Returns float64 [G][D].
+    """
+    q = np.asarray(q_group, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    g, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    n_tok = K.shape[0]
+    sinks = np.arange(min(num_sinks, n_tok))
+    idx = np.asarray(idx, dtype=np.int64)
+    keys = np.concatenate([K[sinks], reconstruct_keys(mu, centroids, code[idx])], axis=0)
+    vals = np.concatenate([V[sinks], V[idx]], axis=0)
+    if keys.shape[0] == 0:
+        return np.zeros((g, d))
+    logits = scale * (q @ keys.T)                                    # [G][T]
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ vals
+
+
+def decode_step(q_group, K, V, mu, centroids, code, k, num_sinks=DEFAULT_SINKS, scale=None):
+    """One decode step of one (sequence, KV head): score, select, attend.
+
+    Returns (out float64 [G][D], idx ascending, scores, condition scale).
+    """
+    sc, cond = scores(q_group, mu, centroids, code, num_sinks)
+    idx = topk(sc, k, num_sinks)
+    out = sparse_attention(q_group, K, V, mu, centroids, code, idx, num_sinks, scale)
+    return out, idx, sc, cond

@@ -1,0 +1,360 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each ``check_*`` takes the oracle module (or a mutated copy of it) and raises
+AssertionError when the oracle disagrees with something the pages or the
+mathematics fix: a hand-worked example from ``tests/golden``, a closed form,
+an invariant, a brute-force enumeration or a library routine.  The pin tests
+call them on the real oracle; the mutation tests call them on deliberately
+broken copies to show that each plausible mistake is caught by at least one.
+
+Page cited: "Self-Indexing KVCache: Predicting Sparse Attention from
+Compressed Keys" (gist.science summary of paper 2603.14224), technical summary
+§2.1 items 1-4.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import sikv_inputs as gen
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# exact mean (§2.1 item 1, entropy-aware normalization)
+# --------------------------------------------------------------------------
+
+def check_exact_sum(o):
+    assert o.exact_sum([1e16, 1.0, -1e16]) == 1
+    assert o.exact_sum([2.0 ** 60, 2.0 ** -60, -(2.0 ** 60)]) == Fraction(1, 2 ** 60)
+    rng = np.random.default_rng(11)
+    for _ in range(20):
+        v = rng.standard_normal(50) * np.exp2(rng.integers(-40, 40, size=50))
+        assert o.exact_sum(v) == sum(Fraction(float(x)) for x in v)
+
+
+def check_round_to_f32(o):
+    one = Fraction(1)
+    ulp = Fraction(1, 2 ** 23)
+    # exact midpoints round to the even neighbour
+    assert o.round_to_f32(one + ulp / 2) == np.float32(1.0)
+    assert o.round_to_f32(one + 3 * ulp / 2) == np.float32(1.0 + 2.0 ** -22)
+    # just above a midpoint rounds up even where a double rounding would not
+    assert o.round_to_f32(one + ulp / 2 + Fraction(1, 2 ** 80)) == np.float32(1.0 + 2.0 ** -23)
+    rng = np.random.default_rng(12)
+    for x in rng.standard_normal(200) * 1e3:
+        assert o.round_to_f32(Fraction(float(x))) == np.float32(x)
+
+
+def check_channel_mean(o):
+    rng = np.random.default_rng(13)
+    for n, s in ((5, 0), (37, 3), (200, 64)):
+        K = rng.standard_normal((n, 8)) * np.exp2(rng.integers(-30, 30, size=(n, 8)))
+        K = K.astype(np.float32).astype(np.float64)
+        mu = o.channel_mean(K, s)
+        rows = K[s:]
+        for c in range(8):
+            want = sum(Fraction(float(x)) for x in rows[:, c]) / rows.shape[0]
+            # brute-force correct rounding: nearest fp32 by enumeration of neighbours
+            cand = np.float32(float(want))
+            nb = [np.nextafter(cand, np.float32(-np.inf)), cand, np.nextafter(cand, np.float32(np.inf))]
+            dist = [abs(Fraction(float(x)) - want) for x in nb]
+            best = min(dist)
+            ok = [np.float32(x) for x, dd in zip(nb, dist) if dd == best]
+            assert mu[c] in ok, (n, s, c, mu[c], ok)
+        # sinks never enter the mean
+        K2 = K.copy()
+        K2[:s] = 1e30
+        assert np.array_equal(o.channel_mean(K2, s), mu)
+    # cancellation that plain fp64 summation gets wrong
+    col = np.array([2.0 ** 60, 3.0, -(2.0 ** 60), 0.0])
+    K = np.stack([col] * 4, axis=1)
+    assert np.all(o.channel_mean(K, 0) == np.float32(0.75))
+    # nothing to average
+    assert np.all(o.channel_mean(np.ones((3, 4)), 64) == 0)
+
+
+# --------------------------------------------------------------------------
+# sign codes and packing (§2.1 items 1 and 3)
+# --------------------------------------------------------------------------
+
+def check_sign_codes_golden(o):
+    g = _load("sign_codes_d8.json")
+    K = np.asarray(g["keys"], dtype=np.float32).astype(np.float64)
+    mu = np.asarray(g["mu"], dtype=np.float32)
+    code = o.sign_codes(K, mu)
+    assert code.tolist() == g["codes"], code.tolist()
+    assert o.pack_codes(code).tolist() == g["packed"]
+
+
+def check_codes_by_construction(o):
+    rng = np.random.default_rng(14)
+    n, d = 64, 32
+    want = rng.integers(0, 16, size=(n, d // 4))
+    mu = rng.standard_normal(d).astype(np.float32)
+    K = np.empty((n, d))
+    for t in range(n):
+        for s in range(d // 4):
+            for i in range(4):
+                bit = (int(want[t, s]) >> i) & 1
+                mag = float(rng.uniform(0.01, 3.0))
+                K[t, 4 * s + i] = float(mu[4 * s + i]) + (mag if bit else -mag)
+    code = o.sign_codes(K.astype(np.float32).astype(np.float64), mu)
+    assert np.array_equal(code, want)
+    packed = o.pack_codes(code)
+    for t in range(n):
+        for m in range(d // 8):
+            assert packed[t, m] == int(want[t, 2 * m]) + 16 * int(want[t, 2 * m + 1])
+    assert np.array_equal(o.unpack_codes(packed), want)
+
+
+# --------------------------------------------------------------------------
+# codebook (§2.1 item 1: one-pass sign-pattern clustering)
+# --------------------------------------------------------------------------
+
+def check_codebook_golden(o):
+    g = _load("codebook_d4.json")
+    for case in g["cases"]:
+        K = np.asarray(case["keys"], dtype=np.float64)
+        s = case["num_sinks"]
+        mu = o.channel_mean(K, s)
+        assert mu.tolist() == case["mu"], (case["name"], mu)
+        code = o.sign_codes(K, mu)
+        assert code.tolist() == case["codes"], (case["name"], code.tolist())
+        cent, counts = o.codebook(K, mu, code, s)
+        want = np.zeros((1, 16, 4))
+        for j, v in case["centroids_nonzero"].items():
+            want[0, int(j)] = v
+        wc = np.zeros((1, 16), dtype=np.int64)
+        for j, v in case["counts_nonzero"].items():
+            wc[0, int(j)] = v
+        assert np.array_equal(cent, want), (case["name"], cent)
+        assert np.array_equal(counts, wc)
+
+
+def check_codebook_invariants(o):
+    w = gen.small(0, n=1500)
+    hi = gen.head_inputs(w, 0, 0)
+    K = gen.storage_to_f64(hi.keys, w.dtype)
+    mu, code, cent, counts = o.encode_keys(K, w.num_sinks)
+    n = K.shape[0] - w.num_sinks
+    assert np.all(counts.sum(axis=1) == n)
+    for s in range(cent.shape[0]):
+        for j in range(16):
+            if counts[s, j] == 0:
+                assert np.all(cent[s, j] == 0)
+                continue
+            for i in range(4):
+                # members all satisfy k >= mu exactly when bit i is set
+                if (j >> i) & 1:
+                    assert cent[s, j, i] >= 0
+                else:
+                    assert cent[s, j, i] < 0
+    # count-weighted centroids add up to the total normalized mass
+    x = K[w.num_sinks:] - mu.astype(np.float64)[None, :]
+    tot = (counts[:, :, None] * cent).sum(axis=1).reshape(-1)
+    assert np.allclose(tot, x.sum(axis=0), rtol=1e-9, atol=1e-6)
+    # cluster membership recounted by brute force
+    for s in (0, 7, 31):
+        for j in (0, 5, 15):
+            assert counts[s, j] == int(np.sum(code[w.num_sinks:, s] == j))
+
+
+def _distinct_pattern_keys(num_sinks: int, d: int = 8, seed: int = 15):
+    """16 non-sink keys whose sub-vectors take each sign pattern once.
+
+    Magnitudes are +-a_i per dimension, so the channel mean is the centre c
+    exactly and every cluster holds one token: reconstruction is exact.
+    """
+    rng = np.random.default_rng(seed)
+    c = rng.integers(-8, 8, size=d).astype(np.float64)
+    a = rng.integers(1, 5, size=d).astype(np.float64)
+    perms = [rng.permutation(16) for _ in range(d // 4)]
+    rows = []
+    for t in range(16):
+        row = np.empty(d)
+        for s in range(d // 4):
+            j = perms[s][t]
+            for i in range(4):
+                row[4 * s + i] = c[4 * s + i] + (a[4 * s + i] if (j >> i) & 1 else -a[4 * s + i])
+        rows.append(row)
+    sinks = rng.standard_normal((num_sinks, d)) * 3
+    return np.concatenate([sinks, np.asarray(rows)], axis=0), c
+
+
+def check_one_member_clusters_reconstruct(o):
+    for s in (0, 3):
+        K, c = _distinct_pattern_keys(s)
+        mu, code, cent, counts = o.encode_keys(K, s)
+        assert np.array_equal(mu, c.astype(np.float32))
+        assert np.all(counts == 1)
+        k_hat = o.reconstruct_keys(mu, cent, code)
+        assert np.array_equal(k_hat[s:], K[s:])
+
+
+# --------------------------------------------------------------------------
+# LUT-GEMV scores (§2.1 item 2)
+# --------------------------------------------------------------------------
+
+def check_scores_golden(o):
+    case = _load("codebook_d4.json")["cases"][0]
+    K = np.asarray(case["keys"], dtype=np.float64)
+    s = case["num_sinks"]
+    mu, code, cent, _ = o.encode_keys(K, s)
+    q = np.asarray(case["queries"])
+    q_bar = o.group_query(q)
+    assert float(np.dot(q_bar, mu.astype(np.float64))) == case["q_bar_dot_mu"]
+    table = o.lut(q_bar, cent)
+    want = np.zeros(16)
+    for j, v in case["lut_nonzero"].items():
+        want[int(j)] = v
+    assert np.array_equal(table[0], want), table
+    sc, cond = o.scores(q, mu, cent, code, s)
+    exp = [(-np.inf if v is None else v) for v in case["scores"]]
+    assert sc.tolist() == exp, sc
+
+
+def check_lut_identity(o):
+    """sum_s LUT[s][code_s] + q_bar.mu = q_bar . k_hat  (identity behind §2.1 item 2)."""
+    w = gen.small(1, n=900, batch=1, num_q_heads=4, num_kv_heads=1)
+    hi = gen.head_inputs(w, 0, 0)
+    K = gen.storage_to_f64(hi.keys, w.dtype)
+    q = gen.storage_to_f64(hi.queries[0], w.dtype)
+    mu, code, cent, _ = o.encode_keys(K, w.num_sinks)
+    sc, cond = o.scores(q, mu, cent, code, w.num_sinks)
+    # independent formulation: dequantize each key coordinate, then a plain dot
+    k_hat = np.empty_like(K)
+    for t in range(K.shape[0]):
+        for dim in range(K.shape[1]):
+            k_hat[t, dim] = float(mu[dim]) + cent[dim // 4, code[t, dim // 4], dim % 4]
+    direct = k_hat @ q.sum(axis=0)
+    sl = slice(w.num_sinks, None)
+    assert np.all(np.abs(sc[sl] - direct[sl]) <= 1e-12 * cond[sl])
+    assert np.all(np.isneginf(sc[:w.num_sinks]))
+    # GQA: the group score is the sum of the single-head scores
+    per_head = sum(o.scores(q[h:h + 1], mu, cent, code, w.num_sinks)[0][sl] for h in range(q.shape[0]))
+    assert np.allclose(per_head, sc[sl], rtol=0, atol=1e-10 * float(cond.max()))
+
+
+# --------------------------------------------------------------------------
+# top-k (selection of the k highest compressed-domain scores)
+# --------------------------------------------------------------------------
+
+def _is_topk_by_definition(score, chosen, k, s):
+    n = len(score)
+    chosen = set(int(t) for t in chosen)
+    if len(chosen) != k or any(t < s or t >= n for t in chosen):
+        return False
+
+    def before(a, b):
+        return score[a] > score[b] or (score[a] == score[b] and a < b)
+
+    for t in chosen:
+        for u in range(s, n):
+            if u not in chosen and not before(t, u):
+                return False
+    return True
+
+
+def check_topk(o):
+    case = _load("codebook_d4.json")["cases"][0]
+    sc = np.array([(-np.inf if v is None else v) for v in case["scores"]])
+    for k, want in case["topk"].items():
+        assert o.topk(sc, int(k), case["num_sinks"]).tolist() == want
+    rng = np.random.default_rng(16)
+    for trial in range(60):
+        n = int(rng.integers(1, 24))
+        s = int(rng.integers(0, min(n, 5) + 1))
+        score = rng.integers(-3, 4, size=n).astype(np.float64)   # many exact ties
+        score[rng.random(n) < 0.2] = -0.0
+        k = int(rng.integers(0, n - s + 1))
+        got = o.topk(score, k, s)
+        assert list(got) == sorted(got)
+        assert _is_topk_by_definition(score, got, k, s), (score, s, k, got)
+
+
+# --------------------------------------------------------------------------
+# sparse attention (§2.1 items 3 and 4)
+# --------------------------------------------------------------------------
+
+def check_attention_golden(o):
+    case = _load("codebook_d4.json")["cases"][0]
+    K = np.asarray(case["keys"], dtype=np.float64)
+    V = np.asarray(case["values"], dtype=np.float64)
+    s = case["num_sinks"]
+    mu, code, cent, _ = o.encode_keys(K, s)
+    q = np.asarray(case["queries"])
+    out = o.sparse_attention(q, K, V, mu, cent, code, np.array([1, 2]), s)
+    assert np.allclose(out, case["attention_k2"]["out"], rtol=0, atol=1e-15), out
+    e = math.e
+    assert np.allclose(out[0], np.array([1, e, 1, 0]) / (2 + e), rtol=0, atol=1e-15)
+
+
+def check_attention_full_selection_is_dense(o):
+    """k = N - S with exact reconstruction equals dense softmax attention over K itself."""
+    import torch
+
+    for s in (0, 2):
+        K, _ = _distinct_pattern_keys(s, seed=17)
+        rng = np.random.default_rng(18)
+        V = rng.standard_normal(K.shape)
+        q = rng.standard_normal((3, K.shape[1]))
+        mu, code, cent, _ = o.encode_keys(K, s)
+        idx = np.arange(s, K.shape[0])
+        out = o.sparse_attention(q, K, V, mu, cent, code, idx, s)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None, :, None, :], torch.from_numpy(K)[None, None].expand(1, 3, -1, -1),
+            torch.from_numpy(V)[None, None].expand(1, 3, -1, -1))[0, :, 0].numpy()
+        assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def check_attention_invariants(o):
+    w = gen.small(0, n=400)
+    hi = gen.head_inputs(w, 0, 0)
+    K = gen.storage_to_f64(hi.keys, w.dtype)
+    V = gen.storage_to_f64(hi.values, w.dtype)
+    mu, code, cent, _ = o.encode_keys(K, w.num_sinks)
+    # no sinks, one selected token: the output is that token's value row
+    out = o.sparse_attention(np.ones((1, 128)), K, V, mu, cent, code, np.array([123]), 0)
+    assert np.allclose(out[0], V[123], rtol=0, atol=1e-12)
+    # a zero query averages the value rows of sinks + selected uniformly
+    idx = np.array([70, 80, 399])
+    out = o.sparse_attention(np.zeros((2, 128)), K, V, mu, cent, code, idx, w.num_sinks)
+    rows = np.concatenate([V[:w.num_sinks], V[idx]])
+    assert np.allclose(out, rows.mean(axis=0)[None, :].repeat(2, 0), rtol=0, atol=1e-12)
+    # selection order does not matter
+    a = o.sparse_attention(np.ones((1, 128)), K, V, mu, cent, code, idx, w.num_sinks)
+    b = o.sparse_attention(np.ones((1, 128)), K, V, mu, cent, code, idx[::-1], w.num_sinks)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+
+
+def check_needle_recall(o):
+    """Planted needle keys are recalled by the compressed-domain selection."""
+    w = gen.config(0)
+    hi = gen.head_inputs(w, 0, 0)
+    K = gen.storage_to_f64(hi.keys, w.dtype)
+    q = gen.storage_to_f64(hi.queries[0], w.dtype)
+    mu, code, cent, _ = o.encode_keys(K, w.num_sinks)
+    sc, _ = o.scores(q, mu, cent, code, w.num_sinks)
+    idx = o.topk(sc, w.topk[0], w.num_sinks)
+    assert set(hi.needle_pos.tolist()) <= set(idx.tolist())
+
+
+ALL_CHECKS = [
+    check_exact_sum, check_round_to_f32, check_channel_mean, check_sign_codes_golden,
+    check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
+    check_one_member_clusters_reconstruct, check_scores_golden, check_lut_identity,
+    check_topk, check_attention_golden, check_attention_full_selection_is_dense,
+    check_attention_invariants, check_needle_recall,
+]
