@@ -1,0 +1,207 @@
+/*
+ * sikv.h -- C ABI of libsikv, the Self-Indexing KVCache decode hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "Self-Indexing KVCache: Predicting Sparse Attention from Compressed
+ * Keys" (summary page at gist.science, paper 2603.14224), technical summary,
+ * cited below as [SIKV 2.1.n] for item n of its section 2.1 (core components):
+ *   2.1.1  sign-based 1-bit vector quantization of the keys: channel-mean
+ *          ("entropy-aware") normalization, 4-dim sub-vectors whose sign
+ *          pattern picks one of 16 clusters, a codebook built in one pass;
+ *          the code both reconstructs the key and indexes it for retrieval;
+ *   2.1.2  compressed-domain top-k retrieval by LUT-GEMV: the query is split
+ *          like the key, each sub-query is dotted with the 16 centroids of its
+ *          subspace, and a token's score sums the table entries its codes pick;
+ *   2.1.3  token-wise code layout (random access per token) and 64
+ *          full-precision sink tokens kept from prefill;
+ *   2.1.4  dequantization fused with the sparse attention pass.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates device memory and keeps no global mutable state.  Every
+ *    call only enqueues kernels on `stream` and returns without synchronizing.
+ *  - Scratch memory comes from the caller's `workspace` (device, 256-byte
+ *    aligned, at least sikv_*_workspace_size() bytes).  The first 256 bytes
+ *    hold a sticky device status word; zero them once before first use
+ *    (sikv_workspace_init) and read them with sikv_check_device_status.
+ *  - Layouts (row-major, contiguous), with B = batch, Hq / Hkv = query / KV
+ *    heads, G = Hq / Hkv (query heads per KV head; query head h*G+g belongs to
+ *    KV head h), D = head_dim = 128, P = D/4 = 32 subspaces, Nmax =
+ *    max_seq_len, S = num_sinks, kmax = max_topk:
+ *      K, V       [B][Hkv][Nmax][D]      dtype (fp32 or bf16)
+ *      q, out     [B][Hq][D]             dtype
+ *      mu         [B][Hkv][D]            fp32   channel means
+ *      codes      [B][Hkv][Nmax][D/8]    uint8  16 bytes per token
+ *      codebook   [B][Hkv][P][16][4]     fp32   centroids of k - mu
+ *      counts     [B][Hkv][P][16]        int32  cluster sizes
+ *      scores     [B][Hkv][Nmax]         fp32
+ *      idx        [B][Hkv][kmax]         int32  selected token positions
+ *      seq_lens   [B]                    int32  N_b, 0 <= N_b <= Nmax (device)
+ *      k_per_seq  [B]                    int32  k_b, 0 <= k_b <= min(kmax, max(N_b - S, 0)) (device)
+ *    Rows past N_b are neither read nor written.
+ *  - Sinks are tokens [0, min(S, N_b)).  Tokens [S, N_b) are the scored,
+ *    "compressed" tokens; n_b = max(N_b - S, 0) of them.
+ *  - Code byte m of a token holds the code of subspace 2m in its low nibble
+ *    and of subspace 2m+1 in its high nibble; bit i of a code is
+ *    [k[4s+i] >= mu[4s+i]] (a tie gives 1).
+ *  - Host-side argument errors return a status and launch nothing.  Errors
+ *    that only the device can see (a seq_len, k or index out of range) set a
+ *    bit of the device status word (SIKV_DEVERR_*), and the offending unit of
+ *    work is skipped; kernels never trap.
+ */
+#ifndef SIKV_H
+#define SIKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SIKV_API __attribute__((visibility("default")))
+#else
+#define SIKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *sikv_stream_t;
+
+typedef enum sikv_status {
+    SIKV_OK = 0,
+    SIKV_ERR_INVALID_ARG = 1,   /* null pointer, bad shape or size */
+    SIKV_ERR_UNSUPPORTED = 2,   /* head_dim != 128, group > 8, unknown dtype, misalignment */
+    SIKV_ERR_WORKSPACE = 3,     /* workspace null, misaligned or too small */
+    SIKV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    SIKV_ERR_DEVICE = 5         /* the device status word holds an error */
+} sikv_status;
+
+typedef enum sikv_dtype {
+    SIKV_DTYPE_F32 = 0,
+    SIKV_DTYPE_BF16 = 1
+} sikv_dtype;
+
+/* Bits of the device status word. */
+#define SIKV_DEVERR_SEQ_LEN 0x1   /* seq_lens[b] < 0 or > max_seq_len */
+#define SIKV_DEVERR_TOPK 0x2      /* k_per_seq[b] < 0, > max_topk or > max(N_b - S, 0) */
+#define SIKV_DEVERR_INDEX 0x4     /* a selected index outside [S, N_b) */
+
+typedef struct sikv_params {
+    int32_t dtype;          /* sikv_dtype of K, V, q and out */
+    int32_t batch;          /* B >= 1 */
+    int32_t num_q_heads;    /* Hq, a multiple of num_kv_heads */
+    int32_t num_kv_heads;   /* Hkv >= 1; G = Hq / Hkv must be <= 8 */
+    int32_t head_dim;       /* D; only 128 is supported */
+    int32_t max_seq_len;    /* Nmax >= 1: row capacity of K, V, codes, scores */
+    int32_t num_sinks;      /* S >= 0 (the pages keep 64) */
+    int32_t max_topk;       /* kmax >= 0: row capacity of idx */
+    float softmax_scale;    /* <= 0 selects 1/sqrt(D) */
+    int32_t reserved[3];    /* must be 0 */
+} sikv_params;
+
+/* Library version as 10000*major + 100*minor + patch. */
+SIKV_API int32_t sikv_version(void);
+
+/* Human-readable name of a status code (static storage). */
+SIKV_API const char *sikv_status_string(sikv_status status);
+
+/* Zero the workspace header (status word); enqueued on `stream`. */
+SIKV_API sikv_status sikv_workspace_init(void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+
+/* Synchronize `stream`, copy the device status word to *device_flags (may be
+ * NULL) and clear it.  Returns SIKV_ERR_DEVICE if any flag was set. */
+SIKV_API sikv_status sikv_check_device_status(void *workspace, size_t workspace_bytes,
+                                     sikv_stream_t stream, int32_t *device_flags);
+
+/* Workspace bytes each entry point needs for these parameters (0 on bad params). */
+SIKV_API size_t sikv_encode_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_score_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_topk_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_sparse_attn_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_decode_workspace_size(const sikv_params *p);
+
+/* Number of kernels one sikv_decode call enqueues for these parameters
+ * (0 on bad params). */
+SIKV_API int32_t sikv_decode_launches(const sikv_params *p);
+
+/*
+ * sikv_encode_keys -- prefill encoder [SIKV 2.1.1, 2.1.3].
+ *
+ * For every (b, h):
+ *   mu[c]       = mean of K[t][c] over t in [S, N_b), computed exactly and
+ *                 rounded once to fp32 (0 when N_b <= S);
+ *   codes[t]    = packed sign-pattern codes of every token t in [0, N_b)
+ *                 (sink rows are written too and never used);
+ *   codebook    = c[s][j] = mean over t in [S, N_b) with code_s(t) == j of
+ *                 K[t][4s:4s+4] - mu[4s:4s+4]; 0 for an empty cluster;
+ *   counts      = cluster sizes (optional output, may be NULL).
+ * Inputs: K (dtype), seq_lens.  Outputs: mu, codes, codebook, counts.
+ */
+SIKV_API sikv_status sikv_encode_keys(const sikv_params *p, const void *K, const int32_t *seq_lens,
+                             float *mu, uint8_t *codes, float *codebook, int32_t *counts,
+                             void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * sikv_score -- compressed-domain LUT-GEMV scoring [SIKV 2.1.2].
+ *
+ * For every (b, h): q_bar = sum of the G query rows of the group;
+ * LUT[s][j] = q_bar[4s:4s+4] . c[s][j]; scores[t] = sum_s LUT[s][code_s(t)]
+ * + q_bar . mu for t in [S, N_b), and -inf for t in [0, min(S, N_b)).
+ * Computed in fp32.  Inputs: q, codes, codebook, mu, seq_lens.
+ */
+SIKV_API sikv_status sikv_score(const sikv_params *p, const void *q, const uint8_t *codes,
+                       const float *codebook, const float *mu, const int32_t *seq_lens,
+                       float *scores, void *workspace, size_t workspace_bytes,
+                       sikv_stream_t stream);
+
+/*
+ * sikv_topk -- exact top-k of the compressed-domain scores [SIKV 2.1.2].
+ *
+ * For every (b, h): the k_b tokens t in [S, N_b) that come first in the
+ * order (score descending, t ascending); -0.0 equals +0.0.  idx[b][h][0..k_b)
+ * receives them in ascending token order and idx[b][h][k_b..kmax) is set to
+ * -1.  Scores must not be NaN.  Inputs: scores, seq_lens, k_per_seq.
+ */
+SIKV_API sikv_status sikv_topk(const sikv_params *p, const float *scores, const int32_t *seq_lens,
+                      const int32_t *k_per_seq, int32_t *idx, void *workspace,
+                      size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * sikv_sparse_attn -- fused dequantization + sparse attention
+ * [SIKV 2.1.3, 2.1.4].
+ *
+ * For every query head (b, h*G+g), over the token set
+ * T = [0, min(S, N_b)) U idx[b][h][0..k_b):
+ *   logit_t = scale * q . K[t]                 for a sink (stored key),
+ *   logit_t = scale * q . (mu + c[code(t)])    for a selected token;
+ *   out     = sum_t softmax(logit)_t * V[t]    (fp32 accumulation).
+ * Entries of idx are attended as listed (order does not matter; duplicates
+ * count twice); an entry outside [S, N_b) sets SIKV_DEVERR_INDEX and is
+ * skipped.  With an empty T the output row is 0.
+ */
+SIKV_API sikv_status sikv_sparse_attn(const sikv_params *p, const void *q, const void *K, const void *V,
+                             const uint8_t *codes, const float *codebook, const float *mu,
+                             const int32_t *idx, const int32_t *k_per_seq,
+                             const int32_t *seq_lens, void *out, void *workspace,
+                             size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * sikv_decode -- one whole decode step: sikv_score, sikv_topk and
+ * sikv_sparse_attn on the same inputs [SIKV 2.1.2-2.1.4].
+ *
+ * idx_out (may be NULL) receives the selected set as sikv_topk writes it;
+ * scores_out (may be NULL) receives the scores as sikv_score writes them.
+ */
+SIKV_API sikv_status sikv_decode(const sikv_params *p, const void *q, const void *K, const void *V,
+                        const uint8_t *codes, const float *codebook, const float *mu,
+                        const int32_t *seq_lens, const int32_t *k_per_seq, void *out,
+                        int32_t *idx_out, float *scores_out, void *workspace,
+                        size_t workspace_bytes, sikv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIKV_H */

@@ -1,0 +1,271 @@
+"""ctypes binding of libsikv (argument marshalling only).
+
+Every function takes torch tensors that live on a CUDA device, checks that
+their dtype, shape and contiguity match the C ABI documented in
+``include/sikv.h``, and passes raw pointers and sizes to the library.  All the
+work runs in the library's CUDA kernels; there is no CPU path.  A missing
+library is built on first use with nvcc; a missing CUDA device or a failed
+launch raises :class:`SikvError`.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from . import build as _build
+
+SIKV_DTYPE_F32 = 0
+SIKV_DTYPE_BF16 = 1
+
+SIKV_DEVERR_SEQ_LEN = 0x1
+SIKV_DEVERR_TOPK = 0x2
+SIKV_DEVERR_INDEX = 0x4
+
+_STATUS = {0: "SIKV_OK", 1: "SIKV_ERR_INVALID_ARG", 2: "SIKV_ERR_UNSUPPORTED", 3: "SIKV_ERR_WORKSPACE",
+           4: "SIKV_ERR_CUDA", 5: "SIKV_ERR_DEVICE"}
+
+EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_check_device_status",
+            "sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
+            "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
+            "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches")
+
+
+class SikvError(RuntimeError):
+    def __init__(self, status: int, where: str, flags: int = 0):
+        self.status = status
+        self.flags = flags
+        msg = f"{where}: {_STATUS.get(status, status)}"
+        if flags:
+            msg += f" (device flags 0x{flags:x})"
+        super().__init__(msg)
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``sikv_params``."""
+
+    _fields_ = [("dtype", ctypes.c_int32), ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
+                ("num_sinks", ctypes.c_int32), ("max_topk", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("reserved", ctypes.c_int32 * 3)]
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def segments(self) -> int:
+        return self.batch * self.num_kv_heads
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == SIKV_DTYPE_F32 else torch.bfloat16
+
+
+def make_params(dtype, batch, num_q_heads, num_kv_heads, max_seq_len, num_sinks=64, max_topk=0,
+                head_dim=128, softmax_scale=0.0) -> Params:
+    if isinstance(dtype, str):
+        dtype = {"f32": SIKV_DTYPE_F32, "bf16": SIKV_DTYPE_BF16}[dtype]
+    elif isinstance(dtype, torch.dtype):
+        dtype = {torch.float32: SIKV_DTYPE_F32, torch.bfloat16: SIKV_DTYPE_BF16}[dtype]
+    return Params(int(dtype), int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), int(max_seq_len),
+                  int(num_sinks), int(max_topk), float(softmax_scale), (ctypes.c_int32 * 3)(0, 0, 0))
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsikv.so (building it in-tree first if it is missing or stale)."""
+    global _LIB
+    if _LIB is None:
+        if not _build.up_to_date():
+            _build.build()
+        L = ctypes.CDLL(_build.LIB)
+        vp, sz, i32, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
+        pp = ctypes.POINTER(Params)
+        L.sikv_version.restype = i32
+        L.sikv_status_string.restype = ctypes.c_char_p
+        L.sikv_status_string.argtypes = [st]
+        L.sikv_workspace_init.argtypes = [vp, sz, vp]
+        L.sikv_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(i32)]
+        for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
+                  "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size"):
+            getattr(L, n).restype = sz
+            getattr(L, n).argtypes = [pp]
+        L.sikv_decode_launches.restype = i32
+        L.sikv_decode_launches.argtypes = [pp]
+        L.sikv_encode_keys.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_score.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_topk.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_sparse_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_decode.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
+                  "sikv_topk", "sikv_sparse_attn", "sikv_decode"):
+            getattr(L, n).restype = st
+        _LIB = L
+    return _LIB
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def version() -> int:
+    return int(lib().sikv_version())
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+
+def _ptr(t, name, dtype=None, shape=None, device=None, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libsikv has no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SikvError(status, where)
+
+
+class Workspace:
+    """A device workspace (torch allocation) with its header zeroed."""
+
+    def __init__(self, nbytes: int, device, stream=None):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        if self.buf.data_ptr() % 256:
+            raise RuntimeError("workspace allocation is not 256-byte aligned")
+        _check(lib().sikv_workspace_init(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes,
+                                         _stream(stream, self.buf.device)), "sikv_workspace_init")
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+    def check(self, stream=None) -> int:
+        """Synchronize, read and clear the device status word; raise on error."""
+        flags = ctypes.c_int32(0)
+        st = lib().sikv_check_device_status(self.ptr, self.nbytes, _stream(stream, self.buf.device),
+                                            ctypes.byref(flags))
+        if st != 0:
+            raise SikvError(st, "device status", flags.value)
+        return flags.value
+
+
+def workspace_size(kind: str, p: Params) -> int:
+    n = getattr(lib(), f"sikv_{kind}_workspace_size")(ctypes.byref(p))
+    if n == 0:
+        raise SikvError(1, f"sikv_{kind}_workspace_size (invalid parameters)")
+    return int(n)
+
+
+def _ws(kind, p, workspace, device, stream):
+    if workspace is None:
+        workspace = Workspace(workspace_size(kind, p), device, stream)
+    return workspace
+
+
+# ----------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------
+
+def sikv_encode_keys(p: Params, K, seq_lens, mu, codes, codebook, counts=None, workspace=None, stream=None):
+    dev = K.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(K, "K", p.torch_dtype, (B, H, N, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(counts, "counts", torch.int32, (B, H, D // 4, 16), dev, optional=True))
+    ws = _ws("encode", p, workspace, dev, stream)
+    _check(lib().sikv_encode_keys(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_encode_keys")
+    return ws
+
+
+def sikv_score(p: Params, q, codes, codebook, mu, seq_lens, scores, workspace=None, stream=None):
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev),
+            _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(scores, "scores", torch.float32, (B, H, N), dev))
+    ws = _ws("score", p, workspace, dev, stream)
+    _check(lib().sikv_score(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_score")
+    return ws
+
+
+def sikv_topk(p: Params, scores, seq_lens, k_per_seq, idx, workspace=None, stream=None):
+    dev = scores.device
+    B, H, N = p.batch, p.num_kv_heads, p.max_seq_len
+    args = (_ptr(scores, "scores", torch.float32, (B, H, N), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev),
+            _ptr(idx, "idx", torch.int32, (B, H, p.max_topk), dev, optional=p.max_topk == 0))
+    ws = _ws("topk", p, workspace, dev, stream)
+    _check(lib().sikv_topk(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_topk")
+    return ws
+
+
+def sikv_sparse_attn(p: Params, q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
+                     workspace=None, stream=None):
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev),
+            _ptr(idx, "idx", torch.int32, (B, H, p.max_topk), dev, optional=p.max_topk == 0),
+            _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(out, "out", p.torch_dtype, (B, p.num_q_heads, D), dev))
+    ws = _ws("sparse_attn", p, workspace, dev, stream)
+    _check(lib().sikv_sparse_attn(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)),
+           "sikv_sparse_attn")
+    return ws
+
+
+def sikv_decode(p: Params, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out=None,
+                scores_out=None, workspace=None, stream=None):
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev),
+            _ptr(out, "out", p.torch_dtype, (B, p.num_q_heads, D), dev),
+            _ptr(idx_out, "idx_out", torch.int32, (B, H, p.max_topk), dev, optional=True),
+            _ptr(scores_out, "scores_out", torch.float32, (B, H, N), dev, optional=True))
+    ws = _ws("decode", p, workspace, dev, stream)
+    _check(lib().sikv_decode(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_decode")
+    return ws
+
+
+def default_scale(head_dim: int = 128) -> float:
+    return 1.0 / math.sqrt(head_dim)

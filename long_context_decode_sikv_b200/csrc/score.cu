@@ -1,0 +1,79 @@
+// sikv_score: compressed-domain LUT-GEMV scores of every cached token.
+//
+// "Self-Indexing KVCache: Predicting Sparse Attention from Compressed Keys",
+// technical summary §2.1 item 2 (LUT-GEMV retrieval) and item 3 (sinks are
+// not scored).  Grid: (token chunk, segment); each CTA builds the segment's
+// tables in shared memory and streams its chunk of 16-byte code rows.
+#include "score_device.cuh"
+#include "sikv_internal.h"
+
+namespace sikv {
+
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kScoreChunk = 4096;      // tokens per CTA (a multiple of 32)
+constexpr int kScoreUnroll = 4;
+
+template <int DT>
+__global__ void __launch_bounds__(kScoreThreads)
+score_kernel(const void *__restrict__ q, const uint8_t *__restrict__ codes,
+             const float *__restrict__ codebook, const float *__restrict__ mu,
+             const int32_t *__restrict__ seq_lens, int hq, int hkv, int nmax, int num_sinks,
+             float *__restrict__ scores, int32_t *status) {
+    extern __shared__ __align__(16) unsigned char score_smem[];
+    ScoreTables &sh = *reinterpret_cast<ScoreTables *>(score_smem);
+    const int seg = blockIdx.y, b = seg / hkv, h = seg % hkv, group = hq / hkv;
+    const int n_tok = load_seq_len(seq_lens, b, nmax, status);
+    if (n_tok < 0) return;
+    const int t_begin = blockIdx.x * kScoreChunk;
+    if (t_begin >= n_tok) return;
+    const int t_end = min(t_begin + kScoreChunk, n_tok);
+    build_score_tables<DT>(sh, q, codebook, mu, b, h, hq, group, seg);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float qmu = sh.qmu;
+    float *srow = scores + static_cast<size_t>(seg) * nmax;
+    const uint4 *crow = reinterpret_cast<const uint4 *>(codes + static_cast<size_t>(seg) * nmax * kCodeBytes);
+    constexpr int kStride = kScoreWarps * 32;
+    for (int g0 = t_begin + warp * 32; g0 < t_end; g0 += kStride * kScoreUnroll) {
+        uint4 rows[kScoreUnroll];
+#pragma unroll
+        for (int u = 0; u < kScoreUnroll; ++u) {
+            const int t = g0 + u * kStride + lane;
+            rows[u] = (t >= num_sinks && t < t_end) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kScoreUnroll; ++u) {
+            const int t = g0 + u * kStride + lane;
+            if (t < t_end) srow[t] = (t >= num_sinks) ? lut2_score(sh.t2, rows[u], lane, qmu) : -INFINITY;
+        }
+    }
+}
+
+}  // namespace
+
+sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,
+                         const float *codebook, const float *mu, const int32_t *seq_lens,
+                         float *scores, int32_t *status, cudaStream_t stream) {
+    const int segs = p.batch * p.num_kv_heads;
+    const dim3 grid((p.max_seq_len + kScoreChunk - 1) / kScoreChunk, segs);
+    const size_t smem = sizeof(ScoreTables);
+    if (p.dtype == SIKV_DTYPE_BF16) {
+        auto kern = score_kernel<SIKV_DTYPE_BF16>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SIKV_ERR_CUDA;
+        kern<<<grid, kScoreThreads, smem, stream>>>(q, codes, codebook, mu, seq_lens, p.num_q_heads,
+                                                    p.num_kv_heads, p.max_seq_len, p.num_sinks, scores, status);
+    } else {
+        auto kern = score_kernel<SIKV_DTYPE_F32>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SIKV_ERR_CUDA;
+        kern<<<grid, kScoreThreads, smem, stream>>>(q, codes, codebook, mu, seq_lens, p.num_q_heads,
+                                                    p.num_kv_heads, p.max_seq_len, p.num_sinks, scores, status);
+    }
+    return cudaGetLastError() == cudaSuccess ? SIKV_OK : SIKV_ERR_CUDA;
+}
+
+}  // namespace sikv

@@ -1,0 +1,135 @@
+// LUT-GEMV scoring in the compressed domain, device side.
+//
+// "Self-Indexing KVCache: Predicting Sparse Attention from Compressed Keys",
+// technical summary §2.1 item 2: the query is split into 4-dim sub-queries,
+// each is dotted with the 16 centroids of its subspace to form a lookup
+// table, and a token's score is the sum of the entries its codes select.
+//
+// B200 layout of the table.  Two subspaces share a code byte, so the 32
+// per-subspace tables are merged into 16 byte-indexed tables
+//   T2[m][b] = LUT[2m][b & 15] + LUT[2m+1][b >> 4],   m = byte position,
+// which halves the lookups to 16 per token.  A warp scores 32 consecutive
+// tokens, one per lane; at step i lane l reads byte (l + i) mod 16 of its
+// code row (the row is rotated in registers by l mod 16 bytes first) and looks
+// it up in shared word  b * 64 + l + i,  which holds T2[(l + i) mod 16][b].
+// Word l + i sits in bank (l + i) mod 32, distinct for the 32 lanes whatever
+// the code bytes are, so every lookup is one conflict-free wavefront.  The
+// byte address (b << 8) | 4l comes out of a single byte-permute, and 4i is a
+// constant offset: one PRMT + one LDS + one FADD per lookup.  The sum order is
+// fixed by t mod 16, so a token's fp32 score does not depend on which kernel
+// or CTA computes it.
+#pragma once
+
+#include "sikv_common.cuh"
+
+namespace sikv {
+
+constexpr int kT2RowWords = 64;                    // words per byte value (48 used)
+constexpr int kT2Words = 256 * kT2RowWords;        // 64 KB
+
+struct ScoreTables {
+    float t2[kT2Words];                // byte-indexed merged tables
+    float qbar[kHeadDim];              // summed group query
+    float lut[kSubspaces * kClusters]; // LUT[s][j]
+    float qmu;                         // q_bar . mu
+    float pad[3];
+};
+
+// Builds q_bar, LUT, q_bar.mu and T2 for segment (b, h) with the whole CTA.
+// Ends with a __syncthreads().
+template <int DT>
+__device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *__restrict__ q,
+                                                   const float *__restrict__ codebook,
+                                                   const float *__restrict__ mu, int b, int h,
+                                                   int hq, int group, int seg) {
+    constexpr int EB = ElemBytes<DT>::value;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const char *qrow = static_cast<const char *>(q) +
+                       (static_cast<size_t>(b) * hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
+    for (int c = tid; c < kHeadDim; c += nt) {
+        float acc = load1<DT>(qrow, c);
+        for (int g = 1; g < group; ++g) acc += load1<DT>(qrow + static_cast<size_t>(g) * kHeadDim * EB, c);
+        sh.qbar[c] = acc;
+    }
+    __syncthreads();
+    const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
+    for (int e = tid; e < kSubspaces * kClusters; e += nt) {
+        const int s = e >> 4;
+        const float4 c4 = __ldg(cb + e);
+        float v = sh.qbar[4 * s] * c4.x;
+        v = fmaf(sh.qbar[4 * s + 1], c4.y, v);
+        v = fmaf(sh.qbar[4 * s + 2], c4.z, v);
+        v = fmaf(sh.qbar[4 * s + 3], c4.w, v);
+        sh.lut[e] = v;
+    }
+    if (tid < 32) {
+        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mu + static_cast<size_t>(seg) * kHeadDim) + tid);
+        double a = static_cast<double>(sh.qbar[4 * tid]) * m4.x;
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 1]), static_cast<double>(m4.y), a);
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 2]), static_cast<double>(m4.z), a);
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 3]), static_cast<double>(m4.w), a);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+        if (tid == 0) sh.qmu = static_cast<float>(a);
+    }
+    __syncthreads();
+    for (int e = tid; e < 256 * 16; e += nt) {
+        const int byte = e >> 4, m = e & 15;
+        const float v = sh.lut[(2 * m) * kClusters + (byte & 15)] + sh.lut[(2 * m + 1) * kClusters + (byte >> 4)];
+        float *row = sh.t2 + byte * kT2RowWords;
+        row[m] = v;
+        row[m + 16] = v;
+        row[m + 32] = v;
+    }
+    __syncthreads();
+}
+
+// Score of the token whose 16-byte code row is `row`, computed by `lane`
+// (the token index must be congruent to lane modulo 16).
+__device__ __forceinline__ float lut2_score(const float *__restrict__ t2, uint4 row, int lane,
+                                            float qmu) {
+    const int r = lane & 15;
+    uint32_t a0 = row.x, a1 = row.y, a2 = row.z, a3 = row.w;
+    if (r & 4) {
+        const uint32_t t = a0;
+        a0 = a1;
+        a1 = a2;
+        a2 = a3;
+        a3 = t;
+    }
+    if (r & 8) {
+        uint32_t t = a0;
+        a0 = a2;
+        a2 = t;
+        t = a1;
+        a1 = a3;
+        a3 = t;
+    }
+    const uint32_t rb = static_cast<uint32_t>(r & 3);
+    const uint32_t sel = rb * 0x1111u + 0x3210u;
+    const uint32_t w0 = __byte_perm(a0, a1, sel), w1 = __byte_perm(a1, a2, sel);
+    const uint32_t w2 = __byte_perm(a2, a3, sel), w3 = __byte_perm(a3, a0, sel);
+    const uint32_t base = 4u * static_cast<uint32_t>(lane);
+    const char *tb = reinterpret_cast<const char *>(t2);
+#define SIKV_LK(W, I) (*reinterpret_cast<const float *>(tb + __byte_perm((W), base, 0x6504u | (((I) & 3u) << 4)) + 4 * (I)))
+    float acc = SIKV_LK(w0, 0);
+    acc += SIKV_LK(w0, 1);
+    acc += SIKV_LK(w0, 2);
+    acc += SIKV_LK(w0, 3);
+    acc += SIKV_LK(w1, 4);
+    acc += SIKV_LK(w1, 5);
+    acc += SIKV_LK(w1, 6);
+    acc += SIKV_LK(w1, 7);
+    acc += SIKV_LK(w2, 8);
+    acc += SIKV_LK(w2, 9);
+    acc += SIKV_LK(w2, 10);
+    acc += SIKV_LK(w2, 11);
+    acc += SIKV_LK(w3, 12);
+    acc += SIKV_LK(w3, 13);
+    acc += SIKV_LK(w3, 14);
+    acc += SIKV_LK(w3, 15);
+#undef SIKV_LK
+    return acc + qmu;
+}
+
+}  // namespace sikv

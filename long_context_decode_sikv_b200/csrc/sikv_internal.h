@@ -1,0 +1,66 @@
+// Internal declarations of libsikv: workspace layouts and kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sikv.h"
+
+namespace sikv {
+
+struct EncodeLayout {
+    int chunk = 0;          // tokens per CTA
+    int nchunks = 0;        // chunks covering [0, Nmax)
+    size_t mean_part = 0;   // double2 [segs][nchunks][D]
+    size_t cb_part = 0;     // double4 [segs][nchunks][P][16]
+    size_t cnt_part = 0;    // int32   [segs][nchunks][P][16]
+    size_t total = 0;
+};
+
+struct TopkLayout {
+    size_t total = 0;
+};
+
+struct AttnLayout {
+    int split = 0;          // list positions per CTA
+    int nsplit = 0;         // splits covering S + kmax positions
+    size_t part_o = 0;      // float [segs][nsplit][G][D]
+    size_t part_ml = 0;     // float2 [segs][nsplit][G]
+    size_t total = 0;
+};
+
+struct DecodeLayout {
+    size_t scores = 0;      // float [segs][Nmax]
+    size_t idx = 0;         // int32 [segs][kmax]
+    size_t attn = 0;        // base offset of an AttnLayout region
+    AttnLayout a;
+    size_t total = 0;
+};
+
+EncodeLayout encode_layout(const sikv_params &p);
+TopkLayout topk_layout(const sikv_params &p);
+AttnLayout attn_layout(const sikv_params &p, size_t base);
+DecodeLayout decode_layout(const sikv_params &p);
+
+sikv_status launch_encode(const sikv_params &p, const void *K, const int32_t *seq_lens, float *mu,
+                          uint8_t *codes, float *codebook, int32_t *counts, char *ws,
+                          cudaStream_t stream);
+
+sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,
+                         const float *codebook, const float *mu, const int32_t *seq_lens,
+                         float *scores, int32_t *status, cudaStream_t stream);
+
+sikv_status launch_topk(const sikv_params &p, const float *scores, const int32_t *seq_lens,
+                        const int32_t *k_per_seq, int32_t *idx, int32_t *status,
+                        cudaStream_t stream);
+
+sikv_status launch_sparse_attn(const sikv_params &p, const void *q, const void *K, const void *V,
+                               const uint8_t *codes, const float *codebook, const float *mu,
+                               const int32_t *idx, const int32_t *k_per_seq,
+                               const int32_t *seq_lens, void *out, char *ws, size_t attn_base,
+                               int32_t *status, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace sikv

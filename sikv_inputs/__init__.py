@@ -57,9 +57,13 @@ ROLE_INDICES = 7
 
 def f32_to_bf16_bits(x) -> np.ndarray:
     """Round fp32 values to bf16 (nearest, ties to even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    bias = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
-    return ((u + bias) >> np.uint32(16)).astype(np.uint16)
+    u = np.array(x, dtype=np.float32, copy=True, order="C").view(np.uint32)
+    bias = u >> 16
+    bias &= 1
+    bias += 0x7FFF
+    u += bias
+    u >>= 16
+    return u.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b) -> np.ndarray:

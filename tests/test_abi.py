@@ -1,0 +1,98 @@
+"""The C-ABI library loads, exports what include/sikv.h declares, and rejects
+bad arguments on the host before touching the GPU (no CUDA device needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_decode_sikv_b200 as sk
+from long_context_decode_sikv_b200 import _binding as bnd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"SIKV_API\s+[^;(]*?\b(sikv_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    decl = _declared()
+    assert {"sikv_encode_keys", "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode"} <= decl
+    lib = sk.lib()
+    for name in sorted(decl):
+        assert hasattr(lib, name), name
+    assert decl <= set(bnd.EXPORTED) | {"sikv_status_string", "sikv_version"}
+
+
+def test_version_and_status_strings():
+    assert sk.version() >= 100
+    for code in range(6):
+        s = sk.lib().sikv_status_string(code).decode()
+        assert s.startswith("SIKV_")
+
+
+def _p(**kw):
+    base = dict(dtype="bf16", batch=2, num_q_heads=8, num_kv_heads=2, max_seq_len=4096, num_sinks=64, max_topk=256)
+    base.update(kw)
+    return sk.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,ok", [
+    ({}, True),
+    ({"head_dim": 64}, False),
+    ({"num_q_heads": 7}, False),
+    ({"num_q_heads": 32, "num_kv_heads": 2}, False),      # group 16 > 8
+    ({"batch": 0}, False),
+    ({"max_seq_len": 0}, False),
+    ({"num_sinks": -1}, False),
+    ({"max_topk": -1}, False),
+    ({"dtype": 7}, False),
+])
+def test_workspace_size_validates_params(kw, ok):
+    p = _p(**kw)
+    n = sk.lib().sikv_decode_workspace_size(ctypes.byref(p))
+    assert (n > 0) == ok
+
+
+def test_workspace_sizes_grow_with_shape():
+    small, big = _p(), _p(max_seq_len=65536, max_topk=4096)
+    for kind in ("sparse_attn", "decode"):
+        assert sk.workspace_size(kind, big) > sk.workspace_size(kind, small) >= 256
+    assert sk.workspace_size("encode", big) >= sk.workspace_size("encode", small) > 256
+
+
+def test_host_rejects_bad_arguments_without_launch():
+    """Null pointers, unsupported shapes and short workspaces return a status."""
+    lib = sk.lib()
+    p = _p()
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+    st = lib.sikv_score(ctypes.byref(p), null, fake, fake, fake, fake, fake, fake, 1 << 20, null)
+    assert st == 1                             # SIKV_ERR_INVALID_ARG
+    bad = _p(head_dim=64)
+    st = lib.sikv_score(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, fake, 1 << 20, null)
+    assert st == 2                             # SIKV_ERR_UNSUPPORTED
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    st = lib.sikv_score(ctypes.byref(p), mis, fake, fake, fake, fake, fake, fake, 1 << 20, null)
+    assert st == 2                             # misaligned q
+    st = lib.sikv_decode(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, null, null,
+                         fake, 1024, null)
+    assert st == 3                             # SIKV_ERR_WORKSPACE (too small)
+    st = lib.sikv_encode_keys(ctypes.byref(p), fake, fake, fake, fake, fake, null,
+                              ctypes.c_void_p((1 << 20) + 16), 1 << 30, null)
+    assert st == 3                             # workspace not 256-byte aligned
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    p = _p()
+    with pytest.raises(ValueError, match="CUDA"):
+        sk.sikv_topk(p, torch.zeros(2, 2, 4096), torch.zeros(2, dtype=torch.int32),
+                     torch.zeros(2, dtype=torch.int32), torch.zeros(2, 2, 256, dtype=torch.int32))
