@@ -26,13 +26,13 @@ constexpr int kSplit = 128;            // list positions per CTA (== threads)
 
 template <int G>
 struct AttnSmem {
-    float qs[G][kHeadDim];
-    float lut[G][kSubspaces * kClusters];
-    float qmu[G];
-    float logit[G][kSplit];
-    int32_t tok[kSplit];
-    float ml[G][2];
-    float red[kAttnWarps][G][kHeadDim];
+    alignas(16) float qs[G][kHeadDim];
+    alignas(16) float lut[G][kSubspaces * kClusters];
+    alignas(16) float qmu[G];
+    alignas(16) float logit[G][kSplit];
+    alignas(16) int32_t tok[kSplit];
+    alignas(16) float ml[G][2];
+    alignas(16) float red[kAttnWarps][G][kHeadDim];   // written with float4 stores
 };
 
 template <int DT, int G>
