@@ -200,6 +200,37 @@ SIKV_API sikv_status sikv_decode(const sikv_params *p, const void *q, const void
                         int32_t *idx_out, float *scores_out, void *workspace,
                         size_t workspace_bytes, sikv_stream_t stream);
 
+/*
+ * sikv_sparse_attn_static -- sikv_sparse_attn for callers that cannot
+ * allocate device memory.  The paper has no counterpart: it is a deployment
+ * variant of the attention step.
+ *
+ * Some callers cannot call cudaMalloc, so they cannot hand the library a
+ * workspace: a serving engine that carves up device memory once at start-up
+ * and may not allocate inside its decode loop, or a plugin host that passes a
+ * kernel only its input and output buffers.  This call computes exactly what
+ * sikv_sparse_attn computes, with the same arguments minus the workspace; its
+ * scratch (split-k partials and the device status word) lives in an 8 MiB
+ * array compiled into the library, which every GPU that loads the library
+ * holds until the process exits.
+ *  - Limit: the partials, B * Hkv * ceil((S + kmax) / 128) * G * 520 bytes
+ *    plus 256, must fit in 8 MiB; larger sizes return SIKV_ERR_WORKSPACE and
+ *    launch nothing.  Invalid parameters return SIKV_ERR_INVALID_ARG.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array: calls that may overlap on the GPU (on
+ *    different streams, or from different threads) race and must be ordered
+ *    by the caller.
+ *  - device_flags (device int32, may be NULL) receives the SIKV_DEVERR_* bits
+ *    of this call.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ */
+SIKV_API sikv_status sikv_sparse_attn_static(const sikv_params *p, const void *q, const void *K,
+                                             const void *V, const uint8_t *codes, const float *codebook,
+                                             const float *mu, const int32_t *idx, const int32_t *k_per_seq,
+                                             const int32_t *seq_lens, void *out, int32_t *device_flags,
+                                             sikv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,8 @@ _STATUS = {0: "SIKV_OK", 1: "SIKV_ERR_INVALID_ARG", 2: "SIKV_ERR_UNSUPPORTED", 3
 EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_check_device_status",
             "sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
             "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
-            "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches")
+            "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
+            "sikv_sparse_attn_static")
 
 
 class SikvError(RuntimeError):
