@@ -22,9 +22,11 @@
  *    never allocates device memory and keeps no global mutable state.  Every
  *    call only enqueues kernels on `stream` and returns without synchronizing.
  *  - Scratch memory comes from the caller's `workspace` (device, 256-byte
- *    aligned, at least sikv_*_workspace_size() bytes).  The first 256 bytes
- *    hold a sticky device status word; zero them once before first use
- *    (sikv_workspace_init) and read them with sikv_check_device_status.
+ *    aligned, at least sikv_*_workspace_size() bytes).  Zero the whole
+ *    workspace once before first use (sikv_workspace_init): its first 256
+ *    bytes hold a sticky device status word (read and cleared with
+ *    sikv_check_device_status), and sikv_decode keeps per-segment counters
+ *    there that every call leaves at zero again.
  *  - Layouts (row-major, contiguous), with B = batch, Hq / Hkv = query / KV
  *    heads, G = Hq / Hkv (query heads per KV head; query head h*G+g belongs to
  *    KV head h), D = head_dim = 128, P = D/4 = 32 subspaces, Nmax =
@@ -87,6 +89,7 @@ typedef enum sikv_dtype {
 #define SIKV_DEVERR_SEQ_LEN 0x1   /* seq_lens[b] < 0 or > max_seq_len */
 #define SIKV_DEVERR_TOPK 0x2      /* k_per_seq[b] < 0, > max_topk or > max(N_b - S, 0) */
 #define SIKV_DEVERR_INDEX 0x4     /* a selected index outside [S, N_b) */
+#define SIKV_DEVERR_TIMEOUT 0x8   /* a bounded wait between the CTAs of a segment ran out */
 
 typedef struct sikv_params {
     int32_t dtype;          /* sikv_dtype of K, V, q and out */
@@ -107,7 +110,7 @@ SIKV_API int32_t sikv_version(void);
 /* Human-readable name of a status code (static storage). */
 SIKV_API const char *sikv_status_string(sikv_status status);
 
-/* Zero the workspace header (status word); enqueued on `stream`. */
+/* Zero the whole workspace; enqueued on `stream`.  Call once per workspace. */
 SIKV_API sikv_status sikv_workspace_init(void *workspace, size_t workspace_bytes, sikv_stream_t stream);
 
 /* Synchronize `stream`, copy the device status word to *device_flags (may be

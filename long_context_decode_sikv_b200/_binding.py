@@ -24,6 +24,7 @@ SIKV_DTYPE_BF16 = 1
 SIKV_DEVERR_SEQ_LEN = 0x1
 SIKV_DEVERR_TOPK = 0x2
 SIKV_DEVERR_INDEX = 0x4
+SIKV_DEVERR_TIMEOUT = 0x8
 
 _STATUS = {0: "SIKV_OK", 1: "SIKV_ERR_INVALID_ARG", 2: "SIKV_ERR_UNSUPPORTED", 3: "SIKV_ERR_WORKSPACE",
            4: "SIKV_ERR_CUDA", 5: "SIKV_ERR_DEVICE"}

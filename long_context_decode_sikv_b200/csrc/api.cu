@@ -71,7 +71,8 @@ DecodeLayout decode_layout(const sikv_params &p) {
     off = align_up(off + segs * (p.max_topk > 0 ? p.max_topk : 1) * sizeof(int32_t), 256);
     L.attn = off;
     L.a = attn_layout(p, off);
-    L.total = L.a.total;
+    L.fused = L.a.total;
+    L.total = fused_layout(p, L.fused).total;
     return L;
 }
 
@@ -102,7 +103,7 @@ const char *sikv_status_string(sikv_status status) {
 
 sikv_status sikv_workspace_init(void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
     SIKV_TRY(check_ws(workspace, workspace_bytes, kHeaderBytes));
-    return cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SIKV_OK
                : SIKV_ERR_CUDA;
 }
@@ -146,6 +147,7 @@ size_t sikv_decode_workspace_size(const sikv_params *p) {
 
 int32_t sikv_decode_launches(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
+    if (fused_plan(*p).ok) return 1;               // one cooperative kernel
     return 1 + (p->max_topk > 0 ? 1 : 0) + 2;     // score, top-k, attention partials + combine
 }
 
@@ -235,6 +237,10 @@ sikv_status sikv_decode(const sikv_params *p, const void *q, const void *K, cons
     char *ws = static_cast<char *>(workspace);
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const FusedPlan plan = fused_plan(*p);
+    if (plan.ok)
+        return launch_decode_fused(*p, plan, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
+                                   scores_out, ws, L.fused, status, s);
     float *sc = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores);
     int32_t *ix = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     SIKV_TRY(launch_score(*p, q, codes, codebook, mu, seq_lens, sc, status, s));

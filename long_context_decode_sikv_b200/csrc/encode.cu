@@ -20,7 +20,8 @@ namespace {
 
 constexpr int kEncThreads = 256;
 constexpr int kEncWarps = kEncThreads / 32;
-constexpr int kEncUnroll = 4;
+constexpr int kEncUnroll = 4;      // rows in flight per thread, mean pass
+constexpr int kEncUnrollCodes = 16; // rows in flight per thread, codes pass (2 CTAs/SM by shared memory)
 
 template <int DT>
 __global__ void __launch_bounds__(kEncThreads)
@@ -139,13 +140,13 @@ enc_codes_partial(const void *__restrict__ K, const int32_t *__restrict__ seq_le
     };
 
     int t = t0 + warp;
-    for (; t + (kEncUnroll - 1) * kEncWarps < t1; t += kEncUnroll * kEncWarps) {
-        float4 v[kEncUnroll];
+    for (; t + (kEncUnrollCodes - 1) * kEncWarps < t1; t += kEncUnrollCodes * kEncWarps) {
+        float4 v[kEncUnrollCodes];
 #pragma unroll
-        for (int u = 0; u < kEncUnroll; ++u)
+        for (int u = 0; u < kEncUnrollCodes; ++u)
             v[u] = load4<DT>(base + static_cast<size_t>(t + u * kEncWarps) * kHeadDim * EB, lane * 4);
 #pragma unroll
-        for (int u = 0; u < kEncUnroll; ++u) consume(t + u * kEncWarps, v[u]);
+        for (int u = 0; u < kEncUnrollCodes; ++u) consume(t + u * kEncWarps, v[u]);
     }
     for (; t < t1; t += kEncWarps)
         consume(t, load4<DT>(base + static_cast<size_t>(t) * kHeadDim * EB, lane * 4));

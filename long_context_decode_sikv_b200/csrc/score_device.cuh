@@ -15,9 +15,9 @@
 // Word l + i sits in bank (l + i) mod 32, distinct for the 32 lanes whatever
 // the code bytes are, so every lookup is one conflict-free wavefront.  The
 // byte address (b << 8) | 4l comes out of a single byte-permute, and 4i is a
-// constant offset: one PRMT + one LDS + one FADD per lookup.  The sum order is
-// fixed by t mod 16, so a token's fp32 score does not depend on which kernel
-// or CTA computes it.
+// constant offset: one PRMT + one LDS + one FADD per lookup.  The sum order
+// (two chains over steps 0-7 and 8-15, then q_bar.mu) is fixed by t mod 16, so
+// a token's fp32 score does not depend on which kernel or CTA computes it.
 #pragma once
 
 #include "sikv_common.cuh"
@@ -30,7 +30,7 @@ constexpr int kT2Words = 256 * kT2RowWords;        // 64 KB
 struct ScoreTables {
     float t2[kT2Words];                // byte-indexed merged tables
     float qbar[kHeadDim];              // summed group query
-    float lut[kSubspaces * kClusters]; // LUT[s][j]
+    float lutT[kClusters * kSubspaces];// LUT[s][j] stored j-major: lutT[j * 32 + s]
     float qmu;                         // q_bar . mu
     float pad[3];
 };
@@ -54,13 +54,13 @@ __device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *
     __syncthreads();
     const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
     for (int e = tid; e < kSubspaces * kClusters; e += nt) {
-        const int s = e >> 4;
-        const float4 c4 = __ldg(cb + e);
+        const int j = e >> 5, s = e & 31;
+        const float4 c4 = __ldg(cb + s * kClusters + j);
         float v = sh.qbar[4 * s] * c4.x;
         v = fmaf(sh.qbar[4 * s + 1], c4.y, v);
         v = fmaf(sh.qbar[4 * s + 2], c4.z, v);
         v = fmaf(sh.qbar[4 * s + 3], c4.w, v);
-        sh.lut[e] = v;
+        sh.lutT[e] = v;
     }
     if (tid < 32) {
         const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mu + static_cast<size_t>(seg) * kHeadDim) + tid);
@@ -73,13 +73,17 @@ __device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *
         if (tid == 0) sh.qmu = static_cast<float>(a);
     }
     __syncthreads();
-    for (int e = tid; e < 256 * 16; e += nt) {
-        const int byte = e >> 4, m = e & 15;
-        const float v = sh.lut[(2 * m) * kClusters + (byte & 15)] + sh.lut[(2 * m + 1) * kClusters + (byte >> 4)];
-        float *row = sh.t2 + byte * kT2RowWords;
-        row[m] = v;
-        row[m + 16] = v;
-        row[m + 32] = v;
+    // One byte value per warp and iteration: lane (m, copy) with m = lane & 15
+    // reads lutT[j * 32 + 2m (+1)] (distinct banks, pairs broadcast) and stores
+    // word m + 16 copy (32 distinct banks), then lanes 0..15 store word m + 32.
+    {
+        const int lane = tid & 31, m = lane & 15, copy = lane >> 4;
+        for (int byte = tid >> 5; byte < 256; byte += nt >> 5) {
+            const float v = sh.lutT[(byte & 15) * kSubspaces + 2 * m] + sh.lutT[(byte >> 4) * kSubspaces + 2 * m + 1];
+            float *row = sh.t2 + byte * kT2RowWords;
+            row[m + 16 * copy] = v;
+            if (copy == 0) row[m + 32] = v;
+        }
     }
     __syncthreads();
 }
@@ -112,24 +116,24 @@ __device__ __forceinline__ float lut2_score(const float *__restrict__ t2, uint4 
     const uint32_t base = 4u * static_cast<uint32_t>(lane);
     const char *tb = reinterpret_cast<const char *>(t2);
 #define SIKV_LK(W, I) (*reinterpret_cast<const float *>(tb + __byte_perm((W), base, 0x6504u | (((I) & 3u) << 4)) + 4 * (I)))
-    float acc = SIKV_LK(w0, 0);
-    acc += SIKV_LK(w0, 1);
-    acc += SIKV_LK(w0, 2);
-    acc += SIKV_LK(w0, 3);
-    acc += SIKV_LK(w1, 4);
-    acc += SIKV_LK(w1, 5);
-    acc += SIKV_LK(w1, 6);
-    acc += SIKV_LK(w1, 7);
-    acc += SIKV_LK(w2, 8);
-    acc += SIKV_LK(w2, 9);
-    acc += SIKV_LK(w2, 10);
-    acc += SIKV_LK(w2, 11);
-    acc += SIKV_LK(w3, 12);
-    acc += SIKV_LK(w3, 13);
-    acc += SIKV_LK(w3, 14);
-    acc += SIKV_LK(w3, 15);
+    // two independent chains (steps 0-7 and 8-15) halve the add latency
+    float a = SIKV_LK(w0, 0), c = SIKV_LK(w2, 8);
+    a += SIKV_LK(w0, 1);
+    c += SIKV_LK(w2, 9);
+    a += SIKV_LK(w0, 2);
+    c += SIKV_LK(w2, 10);
+    a += SIKV_LK(w0, 3);
+    c += SIKV_LK(w2, 11);
+    a += SIKV_LK(w1, 4);
+    c += SIKV_LK(w3, 12);
+    a += SIKV_LK(w1, 5);
+    c += SIKV_LK(w3, 13);
+    a += SIKV_LK(w1, 6);
+    c += SIKV_LK(w3, 14);
+    a += SIKV_LK(w1, 7);
+    c += SIKV_LK(w3, 15);
 #undef SIKV_LK
-    return acc + qmu;
+    return (a + c) + qmu;
 }
 
 }  // namespace sikv

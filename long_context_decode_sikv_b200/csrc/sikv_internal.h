@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "sikv.h"
 
 namespace sikv {
@@ -35,6 +37,7 @@ struct DecodeLayout {
     size_t idx = 0;         // int32 [segs][kmax]
     size_t attn = 0;        // base offset of an AttnLayout region
     AttnLayout a;
+    size_t fused = 0;       // base offset of the fused kernel's coordination region
     size_t total = 0;
 };
 
@@ -60,6 +63,30 @@ sikv_status launch_sparse_attn(const sikv_params &p, const void *q, const void *
                                const int32_t *idx, const int32_t *k_per_seq,
                                const int32_t *seq_lens, void *out, char *ws, size_t attn_base,
                                int32_t *status, cudaStream_t stream);
+
+// Fused single-launch decode (decode_fused.cu).
+constexpr int kFusedMaxCps = 64;          // CTAs per segment, upper bound for the workspace
+
+struct FusedCtl {                          // per-segment counters, zero between launches
+    int arrive1, arrive2, arrive3, ncand;
+    int pad[4];
+};
+
+struct FusedLayout {
+    size_t ghist = 0, ctl = 0, cand = 0, selcnt = 0, part_o = 0, part_ml = 0, total = 0;
+};
+
+struct FusedPlan {
+    bool ok = false;
+    int cps = 0, chunk = 0, npt = 0, gm = 0, grid = 0;
+};
+
+FusedLayout fused_layout(const sikv_params &p, size_t base);
+FusedPlan fused_plan(const sikv_params &p);
+sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
+                                const void *V, const uint8_t *codes, const float *codebook, const float *mu,
+                                const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
+                                float *scores_out, char *ws, size_t base, int32_t *status, cudaStream_t stream);
 
 int device_sm_count();
 

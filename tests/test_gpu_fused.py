@@ -1,0 +1,107 @@
+"""The single-launch decode kernel against the standalone entry points and
+the oracle.
+
+sikv_decode runs one cooperative kernel whenever every CTA of the step fits on
+the device at once.  Its scores must be bit-identical to sikv_score's (same
+table, same order of additions per token), its selection identical to
+sikv_topk's on those scores, and its attention within the attention
+tolerance of sikv_sparse_attn's over that selection.
+"""
+
+import ctypes
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_decode_sikv_b200 as sk
+import oracle
+import sikv_inputs as gen
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = {
+    "two-chunks": lambda: gen.small(1, n=2085, batch=1, num_q_heads=8, num_kv_heads=2),
+    "many-chunks": lambda: replace(gen.config(1), name="many", batch=1, num_q_heads=8, num_kv_heads=2,
+                                   seq_lens=(40000,), topk=(3000,), needles_per_head=8),
+    "ragged-empty-chunks": lambda: gen.small(3, n=9000, batch=4, num_q_heads=8, num_kv_heads=2),
+    "gqa8": lambda: gen.small(2, n=5000, batch=1, num_q_heads=16, num_kv_heads=2),
+    "gqa5": lambda: gen.small(1, n=4100, batch=2, num_q_heads=10, num_kv_heads=2),
+    "f32-one-head": lambda: gen.small(0, n=6000),
+    "k-equals-n": lambda: replace(gen.config(1), name="kn", batch=2, num_q_heads=4, num_kv_heads=1,
+                                  seq_lens=(3000, 2500), topk=(2936, 2436), needles_per_head=2),
+}
+
+
+def _fused_runs(p):
+    return int(sk.lib().sikv_decode_launches(ctypes.byref(p))) == 1
+
+
+def _standalone(dw, step):
+    w, dev, c = dw.w, dw.dev, dw.cache
+    sc = torch.full((w.batch, w.num_kv_heads, w.max_seq_len), 12345.0, device=dev)
+    sk.sikv_score(dw.p, dw.q[step], c.codes, c.codebook, c.mu, dw.seq_lens, sc).check()
+    idx = torch.full((w.batch, w.num_kv_heads, w.max_topk), -7, dtype=torch.int32, device=dev)
+    sk.sikv_topk(dw.p, sc, dw.seq_lens, dw.k, idx).check()
+    out = torch.empty((w.batch, w.num_q_heads, 128), dtype=dw.p.torch_dtype, device=dev)
+    sk.sikv_sparse_attn(dw.p, dw.q[step], dw.K, dw.V, c.codes, c.codebook, c.mu, idx, dw.k, dw.seq_lens,
+                        out).check()
+    return out, idx, sc
+
+
+@pytest.mark.parametrize("name", sorted(SHAPES))
+def test_fused_matches_standalone_entry_points(name):
+    dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1))
+    assert _fused_runs(dw.p), "the single-launch kernel should cover this shape"
+    dw.encode()
+    atol, rtol = gu.attn_tol(dw.w.dtype)
+    for step in (0, 1):
+        out_f, idx_f, sc_f = dw.decode(step=step)
+        out_s, idx_s, sc_s = _standalone(dw, step)
+        for b in range(dw.w.batch):
+            n = dw.w.seq_lens[b]
+            assert torch.equal(sc_f[b, :, :n], sc_s[b, :, :n]), (name, step, b)
+        assert torch.equal(idx_f, idx_s), (name, step)
+        assert np.allclose(gu.to_f64(out_f), gu.to_f64(out_s), atol=atol, rtol=rtol), name
+
+
+def test_fused_repeated_calls_leave_clean_state():
+    """Every call resets the per-segment counters: repeated calls agree bit for bit."""
+    dw = gu.DeviceWorkload(SHAPES["many-chunks"](), steps=(0, 1))
+    dw.encode()
+    first = [t.clone() for t in dw.decode(step=1)]
+    for _ in range(3):
+        dw.decode(step=0)
+        again = dw.decode(step=1)
+        for x, y in zip(first, again):
+            assert torch.equal(x, y)
+
+
+def test_fused_all_scores_tied_takes_lowest_indices():
+    """Identical keys: every score ties, the threshold bin holds every token
+    (the candidate list does not fit in shared memory) and the selection falls
+    back to the lowest token indices."""
+    dev = gu.device()
+    n, k, S = 20000, 1500, 64
+    w = replace(gen.config(1), name="ties", batch=1, num_q_heads=4, num_kv_heads=1, seq_lens=(n,), topk=(k,),
+                needles_per_head=0)
+    rng = np.random.default_rng(5)
+    row = gen.to_storage(rng.standard_normal(128), "bf16")
+    K = np.broadcast_to(row, (1, 1, n, 128)).copy()
+    V = gen.to_storage(rng.standard_normal((1, 1, n, 128)), "bf16")
+    q = gen.to_storage(rng.standard_normal((1, 4, 128)), "bf16")
+    bt = gen.Batch(w, K, V, {0: q}, np.array([n], np.int32), np.array([k], np.int32), None, {(0, 0): np.zeros(0)})
+    dw = gu.DeviceWorkload(w, bt=bt)
+    assert _fused_runs(dw.p)
+    dw.encode()
+    out, idx, sc = dw.decode()
+    Kf = gen.storage_to_f64(K[0, 0], "bf16")
+    Vf = gen.storage_to_f64(V[0, 0], "bf16")
+    qf = gen.storage_to_f64(q[0], "bf16")
+    mu, code, cent, _ = oracle.encode_keys(Kf, S)
+    o_out, o_idx, o_sc, cond = oracle.decode_step(qf, Kf, Vf, mu, cent, code, k, S)
+    assert np.array_equal(o_idx, np.arange(S, S + k))
+    assert np.array_equal(idx[0, 0].cpu().numpy(), o_idx)
+    assert np.allclose(gu.to_f64(out)[0], o_out, atol=2e-2, rtol=1e-2)
