@@ -8,25 +8,30 @@
 //
 // Work split.  Each (sequence, KV head) segment is cut into `cps` chunks of
 // `chunk` tokens, one CTA per chunk, all CTAs co-resident (cooperative
-// launch).  A CTA keeps the scores of its chunk in registers (NPT per thread)
-// and never writes them to memory unless asked to.  The CTAs of a segment
+// launch).  A CTA never writes its scores to memory (unless asked to): it
+// keeps each token's histogram bin in shared memory.  The CTAs of a segment
 // agree on the selection through three counters in the workspace:
-//   1. every CTA builds a 2048-bin histogram of its scores (bins linear in the
+//   1. every CTA builds a 1024-bin histogram of its scores (bins linear in the
 //      score between the bounds the LUT implies, so a higher bin means a
 //      strictly higher score), finds its own local k-th bin b_c and adds its
-//      counts for bins >= b_c into the segment histogram (the global k-th bin
-//      b* is >= every b_c, so the lower bins are never needed);  arrive #1;
+//      counts for bins >= b_c into the segment histogram (the segment's k-th
+//      bin b* is >= every b_c, so the lower bins are never needed);  arrive #1;
 //   2. after all arrivals every CTA scans the segment histogram from the top
 //      and finds b*; tokens in higher bins are selected outright, tokens in
-//      b* are written to a candidate list;  arrive #2;
-//   3. every CTA radix-selects, from the candidates, the exact k-th key T and
-//      the lowest-index ties it needs (the same answer in every CTA), marks its
-//      selected tokens, and attends over them (plus its share of the sinks)
-//      with an online softmax; it writes (m, l, o) partials;  arrive #3 — the
-//      last CTA to arrive merges the partials into the output and zeroes the
-//      segment's coordination state for the next launch.
+//      b* are re-scored and appended with their exact keys to a candidate
+//      list;  arrive #2;
+//   3. every CTA ranks the candidates (order: key descending, token
+//      ascending) and marks the winners of its own chunk — the same answer in
+//      every CTA — then attends over its selected tokens and its share of the
+//      sinks with an online softmax and writes (m, l, o) partials;  arrive #3 —
+//      the last CTA to arrive merges the partials into the output and zeroes
+//      the segment's coordination state for the next launch.
 // Waits are bounded: a wait that runs out sets SIKV_DEVERR_TIMEOUT and the
 // CTA carries on, so a kernel always ends.
+//
+// Code size matters here: every phase but the scoring loop runs once per CTA
+// with a cold instruction cache, so loops over a thread's tokens stay rolled
+// (their state lives in shared memory, not in registers).
 #include "score_device.cuh"
 #include "sikv_internal.h"
 
@@ -36,13 +41,18 @@ namespace {
 
 constexpr int kFT = 256;                 // threads per CTA
 constexpr int kFW = kFT / 32;            // warps per CTA
-constexpr int kFBins = 2048;             // histogram bins per segment
+constexpr int kFBins = 1024;             // histogram bins per segment
 constexpr int kFTile = 256;              // list entries attended per pass
-constexpr int kFCandSmem = 1024;         // candidates staged in shared memory
-constexpr int kFUnroll = 8;              // code rows in flight per thread
 constexpr int kFListCap = 2048;          // attended tokens staged per window
-constexpr int kFGroups = 64 * kFW;       // (register slot, warp) groups, NPT <= 64
+constexpr int kFMaxNpt = 64;             // token slots per thread at most
+constexpr int kFMaxChunk = kFMaxNpt * kFT;
+constexpr int kFCandSmem = 1024;         // candidates staged in shared memory
+constexpr int kFRankMax = 512;           // up to this many candidates: rank directly
+constexpr int kFUnroll = 8;              // code rows in flight per thread
+constexpr int kFPrefetchRows = 16;       // code rows per thread kept ahead in L2
+constexpr int kFVRows = 8;               // value rows in flight per warp
 constexpr int kSpinLimit = 1 << 23;      // ~1 s of __nanosleep(128) polls
+constexpr int kFRow = 256;               // tokens per row scan of a warp (32 lanes x 8)
 
 struct FusedArgs {
     const void *q, *K, *V;
@@ -52,7 +62,7 @@ struct FusedArgs {
     void *out;
     int32_t *idx_out;
     float *scores_out;
-    int hq, hkv, nmax, num_sinks, kmax, cps, chunk, cand_cap;
+    int hq, hkv, nmax, num_sinks, kmax, cps, chunk, npt, cand_cap;
     float scale;
     uint32_t *ghist;      // [segs][kFBins]
     uint2 *cand;          // [segs][cand_cap] (key, token)
@@ -63,26 +73,37 @@ struct FusedArgs {
     int32_t *status;
 };
 
+// Shared memory.  The union is reused in time: scoring tables (until the
+// candidates are written), then the candidate ranking buffers, then the
+// attention buffers.
 template <int GM>
 struct FusedSmem {
     union {
-        ScoreTables tab;                         // scoring phase
+        ScoreTables tab;
         struct {
-            int32_t list[kFListCap];             // ordered tokens to attend (one window)
-            uint32_t grp[kFGroups];              // per-(slot, warp) ordinal bases
+            uint32_t ckey[kFCandSmem];
+            int32_t cidx[kFCandSmem];
+            uint32_t winbits[kFMaxChunk / 32];
+        } sel;
+        struct {
+            int32_t list[kFListCap];
             alignas(16) float logit[GM][kFTile];
             alignas(16) float red[kFW][GM][kHeadDim];
-        } at;                                    // attention phase
+            alignas(16) float luth[kSubspaces * kClusters][GM];   // per-head LUT, [s*16+j][g]
+        } at;
     } u;
     alignas(16) float qs[GM][kHeadDim];
-    alignas(16) float luth[kSubspaces * kClusters][GM];   // per-head LUT, [s*16+j][g]
+    alignas(16) float mus[kHeadDim];
     alignas(16) float qmu_h[GM];
     alignas(16) float run_m[GM];
     alignas(16) float run_l[GM];
     alignas(16) float tile_stat[kFW][GM];
     uint32_t hist[kFBins];
-    uint32_t ckey[kFCandSmem];
-    int32_t cidx[kFCandSmem];
+    // one entry per token of the chunk, in token order (entry p: token t0 + p,
+    // scored by thread p mod 256): its bin + 1 (0: no token), bit 15 set once
+    // the token is selected.  Holds the codebook before scoring.
+    alignas(16) uint16_t bins[kFMaxChunk];
+    uint32_t rowcnt[kFMaxChunk / 256];        // selected tokens per row of 256, then their prefix
     uint32_t wtot[kFW + 1];
     uint32_t sc[16];
     float bin_lo, bin_inv;
@@ -93,6 +114,10 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Thread 0 waits until *ctr >= target (bounded); the CTA then synchronizes.
@@ -148,27 +173,31 @@ __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t *wtot, ui
     return r;
 }
 
-// In a histogram of `nbins` bins scanned from the top bin down, finds the bin
-// where the running count first reaches `need` (1 <= need <= total).  Each
-// thread owns nbins/256 consecutive bins.  Writes (bin, count above) to
-// out[0..1].  Ends synchronized.
-template <typename Load>
-__device__ __forceinline__ void cta_find_bin(Load load, int nbins, uint32_t need, uint32_t *wtot, uint32_t *out) {
-    const int per = nbins / kFT;
-    const int top = nbins - 1 - threadIdx.x * per;
+// In a histogram of PER * 256 bins scanned from the top bin down, finds the
+// bin where the running count first reaches `need` (1 <= need <= total).
+// Each thread loads its PER consecutive bins once.  Writes (bin, count above)
+// to out[0..1]; out is left untouched when the total is below need.  Ends
+// synchronized.
+template <int PER, typename Load>
+__device__ __forceinline__ void cta_find_bin(Load load, uint32_t need, uint32_t *wtot, uint32_t *out) {
+    const int top = PER * kFT - 1 - static_cast<int>(threadIdx.x) * PER;
+    uint32_t h[PER];
     uint32_t loc = 0;
-    for (int i = 0; i < per; ++i) loc += load(top - i);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        h[i] = load(top - i);
+        loc += h[i];
+    }
     uint32_t total;
     uint32_t above = cta_excl_scan(loc, wtot, &total);
     if (above < need && need <= above + loc) {
-        for (int i = 0; i < per; ++i) {
-            const uint32_t h = load(top - i);
-            if (above + h >= need) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            if (above < need && above + h[i] >= need) {
                 out[0] = static_cast<uint32_t>(top - i);
                 out[1] = above;
-                break;
             }
-            above += h;
+            above += h[i];
         }
     }
     __syncthreads();
@@ -178,9 +207,10 @@ __device__ __forceinline__ void cta_find_bin(Load load, int nbins, uint32_t need
 // keep(e)): returns the key of rank `need` counted from the largest and, in
 // *need_left, how many elements equal to it are still needed.  Uses hist[0..255].
 template <typename KeyF, typename KeepF>
-__device__ __forceinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, uint32_t need, uint32_t *hist,
-                                                     uint32_t *wtot, uint32_t *sc, uint32_t *need_left) {
+__device__ __noinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, uint32_t need, uint32_t *hist,
+                                                  uint32_t *wtot, uint32_t *sc, uint32_t *need_left) {
     uint32_t prefix = 0, mask = 0;
+#pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += kFT) hist[i] = 0;
         __syncthreads();
@@ -190,7 +220,7 @@ __device__ __forceinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n
             if (((k ^ prefix) & mask) == 0) atomicAdd(&hist[(k >> shift) & 255u], 1u);
         }
         __syncthreads();
-        cta_find_bin([&](int i) { return hist[i]; }, 256, need, wtot, sc);
+        cta_find_bin<1>([&](int i) { return hist[i]; }, need, wtot, sc);
         prefix |= sc[0] << shift;
         mask |= 255u << shift;
         need -= sc[1];
@@ -200,14 +230,53 @@ __device__ __forceinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n
     return prefix;
 }
 
-// Exact score of token t, recomputed by the lane that scored it (same table,
-// same rotation, same order of additions: bit-identical).  Only tokens in the
-// threshold bin need it, so it stays out of line.
-__device__ __noinline__ float rescore(const float *t2, const uint4 *crow, int t, int lane, float qmu) {
-    return lut2_score(t2, __ldg(crow + t), lane, qmu);
+// Appends token t of the threshold bin to the segment's candidate list with
+// its exact key: re-scored by the lane that scored it (same table, same
+// rotation, same order of additions, so bit-identical).
+__device__ __noinline__ void emit_candidate(const float *t2, const uint4 *crow, int t, int lane, float qmu,
+                                            int *ncand, uint2 *cand, int cap) {
+    const float sv = lut2_score(t2, __ldg(crow + t), lane, qmu);
+    const int slot = atomicAdd(ncand, 1);
+    if (slot < cap) cand[slot] = make_uint2(score_key(sv), static_cast<uint32_t>(t));
 }
 
-template <int DT, int GM, int NPT>
+// bins[] holds one 16-bit entry per token of the chunk in token order (entry
+// p is token t0 + p).  A lane scans 8 consecutive entries with one 16-byte
+// load; these give, per 16-bit half of each word, an all-ones mask where the
+// entry's bin is above / equal to a threshold (entries hold bin + 1).
+__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return __vcmpgtu2(w & 0x7FFF7FFFu, thr2); }
+__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) { return __vcmpeq2(w & 0x7FFF7FFFu, thr2); }
+// 8-bit mask (bit j = entry j of the lane's 8) from four per-half masks
+__device__ __forceinline__ uint32_t mask8(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
+    return (m0 & 1u) | ((m0 >> 15) & 2u) | ((m1 & 1u) << 2) | ((m1 >> 13) & 8u) | ((m2 & 1u) << 4) |
+           ((m2 >> 11) & 32u) | ((m3 & 1u) << 6) | ((m3 >> 9) & 128u);
+}
+
+// Winners among many candidates (more than the rank path takes): radix
+// select of the need-th key and of the lowest tied token indices, then one
+// marking pass.  Returns this thread's count of winners before the chunk.
+// Kept out of line: it only runs for heavily tied or flat score tables.
+__device__ __noinline__ uint32_t refine_by_radix(const uint2 *cand, int ncand, uint32_t need, int t0, int chunk,
+                                                 uint32_t *winbits, uint32_t *hist, uint32_t *wtot, uint32_t *sc) {
+    uint32_t ties_needed, left, before = 0;
+    const uint32_t T = cta_radix_select([&](int e) { return __ldcg(cand + e).x; }, [&](int) { return true; }, ncand,
+                                        need, hist, wtot, sc, &ties_needed);
+    // the ties_needed lowest token indices among keys equal to T
+    const uint32_t tie_idx = ~cta_radix_select([&](int e) { return ~__ldcg(cand + e).y; },
+                                               [&](int e) { return __ldcg(cand + e).x == T; }, ncand, ties_needed,
+                                               hist, wtot, sc, &left);
+    for (int e = threadIdx.x; e < ncand; e += kFT) {
+        const uint2 v = __ldcg(cand + e);
+        if (v.x > T || (v.x == T && v.y <= tie_idx)) {
+            const int rel = static_cast<int>(v.y) - t0;
+            if (rel >= 0 && rel < chunk) atomicOr(&winbits[rel >> 5], 1u << (rel & 31));
+            else if (rel < 0) ++before;
+        }
+    }
+    return before;
+}
+
+template <int DT, int GM>
 __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     constexpr int EB = ElemBytes<DT>::value;
     extern __shared__ __align__(16) unsigned char fused_smem[];
@@ -216,6 +285,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int seg = blockIdx.x / a.cps, c = blockIdx.x % a.cps;
     const int b = seg / a.hkv, h = seg % a.hkv, group = a.hq / a.hkv;
+    const int npt = a.npt;
     FusedCtl *ctl = a.ctl + seg;
 
     // ---- lengths (an invalid segment decodes as empty but still takes part)
@@ -232,165 +302,171 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     }
     const int t0 = c * a.chunk;
     const int t1 = min(t0 + a.chunk, n_tok);
+    const int tstart = max(t0, a.num_sinks);
+    const size_t kv_seg = static_cast<size_t>(seg) * a.nmax;
+    const uint4 *crow = reinterpret_cast<const uint4 *>(a.codes) + kv_seg;
+    const int my = 32 * warp + lane;                         // slot i of this thread: token t0 + 256 i + my
 
-    // ---- tables: byte-indexed scoring tables, per-head LUTs, bounds
-    build_score_tables<DT>(sh.u.tab, a.q, a.codebook, a.mu, b, h, a.hq, group, seg);
-    {
-        const char *qrow = static_cast<const char *>(a.q) +
-                           (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
-        for (int e = tid; e < GM * kHeadDim; e += kFT) {
-            const int g = e / kHeadDim, d = e % kHeadDim;
-            sh.qs[g][d] = g < group ? load1<DT>(qrow + static_cast<size_t>(g) * kHeadDim * EB, d) : 0.f;
-        }
-        for (int i = tid; i < kFBins; i += kFT) sh.hist[i] = 0;
+    // ---- tables.  The prologue leaves HBM idle, so the first code rows and
+    // this CTA's share of the sink rows go to L2 meanwhile.
+#pragma unroll 1
+    for (int i = 0; i < kFPrefetchRows && i < npt; ++i) {
+        const int t = t0 + kFT * i + my;
+        if (t >= tstart && t < t1) prefetch_l2(crow + t);
     }
-    __syncthreads();
     {
-        const float4 *cb = reinterpret_cast<const float4 *>(a.codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
-        for (int e = tid; e < kSubspaces * kClusters * GM; e += kFT) {
-            const int r = e / GM, g = e % GM, s = r >> 4;
-            const float4 c4 = __ldg(cb + r);
-            float v = sh.qs[g][4 * s] * c4.x;
-            v = fmaf(sh.qs[g][4 * s + 1], c4.y, v);
-            v = fmaf(sh.qs[g][4 * s + 2], c4.z, v);
-            v = fmaf(sh.qs[g][4 * s + 3], c4.w, v);
-            sh.luth[r][g] = v;
+        const int n_sinks0 = min(a.num_sinks, n_tok);
+        for (int sk = c + a.cps * tid; sk < n_sinks0; sk += a.cps * kFT) {
+            prefetch_l2(static_cast<const char *>(a.K) + (kv_seg + sk) * kHeadDim * EB);
+            prefetch_l2(static_cast<const char *>(a.V) + (kv_seg + sk) * kHeadDim * EB);
         }
-        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(a.mu + static_cast<size_t>(seg) * kHeadDim) + lane);
-        for (int g = warp; g < GM; g += kFW) {
-            double s = static_cast<double>(sh.qs[g][4 * lane]) * m4.x;
-            s = fma(static_cast<double>(sh.qs[g][4 * lane + 1]), static_cast<double>(m4.y), s);
-            s = fma(static_cast<double>(sh.qs[g][4 * lane + 2]), static_cast<double>(m4.z), s);
-            s = fma(static_cast<double>(sh.qs[g][4 * lane + 3]), static_cast<double>(m4.w), s);
+    }
+    float4 *cbs = reinterpret_cast<float4 *>(sh.bins);     // 8 KB, free until scoring
+    for (int e = tid; e < GM * kHeadDim; e += kFT) sh.qs[e / kHeadDim][e % kHeadDim] = 0.f;
+    __syncthreads();
+    stage_table_inputs<DT>(&sh.qs[0][0], cbs, sh.mus, a.q, a.codebook, a.mu, b, h, a.hq, group, seg);
+    for (int i = tid; i < kFBins; i += kFT) sh.hist[i] = 0;
+    __syncthreads();
+    build_score_tables(sh.u.tab, &sh.qs[0][0], cbs, sh.mus, group);
+    for (int g = warp; g < GM; g += kFW) {
+        double s = static_cast<double>(sh.qs[g][4 * lane]) * sh.mus[4 * lane];
+        s = fma(static_cast<double>(sh.qs[g][4 * lane + 1]), static_cast<double>(sh.mus[4 * lane + 1]), s);
+        s = fma(static_cast<double>(sh.qs[g][4 * lane + 2]), static_cast<double>(sh.mus[4 * lane + 2]), s);
+        s = fma(static_cast<double>(sh.qs[g][4 * lane + 3]), static_cast<double>(sh.mus[4 * lane + 3]), s);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (lane == 0) sh.qmu_h[g] = static_cast<float>(s);
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) sh.qmu_h[g] = static_cast<float>(s);
+    }
+    if (warp == kFW - 1) {
+        // score bounds: q_bar.mu + sum over subspaces of the min / max LUT entry
+        float lo = INFINITY, hi = -INFINITY;
+        for (int j = 0; j < kClusters; ++j) {
+            const float v = sh.u.tab.lutT[j * kSubspaces + lane];
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
         }
-        if (warp == kFW - 1) {
-            // score bounds: q_bar.mu + sum over subspaces of the min / max LUT entry
-            float lo = INFINITY, hi = -INFINITY;
-            for (int j = 0; j < kClusters; ++j) {
-                const float v = sh.u.tab.lutT[j * kSubspaces + lane];
-                lo = fminf(lo, v);
-                hi = fmaxf(hi, v);
-            }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                lo += __shfl_xor_sync(0xffffffffu, lo, off);
-                hi += __shfl_xor_sync(0xffffffffu, hi, off);
-            }
-            if (lane == 0) {
-                lo += sh.u.tab.qmu;
-                hi += sh.u.tab.qmu;
-                const float width = hi - lo;
-                const float inv = static_cast<float>(kFBins) / width;
-                sh.bin_lo = lo;
-                sh.bin_inv = inv;
-                sh.bin_flat = !(isfinite(width) && width > 0.f && isfinite(inv));
-            }
+        for (int off = 16; off > 0; off >>= 1) {
+            lo += __shfl_xor_sync(0xffffffffu, lo, off);
+            hi += __shfl_xor_sync(0xffffffffu, hi, off);
+        }
+        if (lane == 0) {
+            lo += sh.u.tab.qmu;
+            hi += sh.u.tab.qmu;
+            const float width = hi - lo;
+            const float inv = static_cast<float>(kFBins) / width;
+            sh.bin_lo = lo;
+            sh.bin_inv = inv;
+            sh.bin_flat = !(isfinite(width) && width > 0.f && isfinite(inv));
         }
     }
     __syncthreads();
     const float bin_lo = sh.bin_lo, bin_inv = sh.bin_inv;
     const bool bin_flat = sh.bin_flat != 0;
-    auto bin_of = [&](float s) -> int {
-        if (bin_flat) return 0;
-        const int v = __float2int_rz((s - bin_lo) * bin_inv);
-        return min(max(v, 0), kFBins - 1);
-    };
-
-    // ---- scores of this chunk; each thread keeps only the histogram bin of
-    // its tokens (16 bits each, bin + 1, 0 = no token), two per register.
-    // Register slot i of (warp w, lane l) is token t0 + 256 i + 32 w + l.
-    constexpr int NPK = NPT / 2;
-    uint32_t binpk[NPK];
     const float qmu = sh.u.tab.qmu;
-    const uint4 *crow = reinterpret_cast<const uint4 *>(a.codes) + static_cast<size_t>(seg) * a.nmax;
-    const int tstart = max(t0, a.num_sinks);
+
+    // ---- scores of this chunk -> histogram and per-slot bins
     {
-        float *so = a.scores_out ? a.scores_out + static_cast<size_t>(seg) * a.nmax : nullptr;
+        float *so = a.scores_out ? a.scores_out + kv_seg : nullptr;
+#pragma unroll 1
+        for (int i0 = 0; i0 < npt; i0 += kFUnroll) {
 #pragma unroll
-        for (int i = 0; i < NPK; ++i) binpk[i] = 0;
-#pragma unroll
-        for (int i0 = 0; i0 < NPT; i0 += kFUnroll) {
+            for (int u = 0; u < kFUnroll; ++u) {
+                const int t = t0 + kFT * (i0 + kFPrefetchRows + u) + my;
+                if (i0 + kFPrefetchRows + u < npt && t >= tstart && t < t1) prefetch_l2(crow + t);
+            }
             uint4 rows[kFUnroll];
 #pragma unroll
             for (int u = 0; u < kFUnroll; ++u) {
-                const int t = t0 + kFT * (i0 + u) + 32 * warp + lane;
-                rows[u] = (t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
+                const int t = t0 + kFT * (i0 + u) + my;
+                rows[u] = (i0 + u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
             }
-            // keep the next batch's loads below this point: kFUnroll rows in
-            // flight per thread, not the whole unrolled chunk
-            asm volatile("" ::: "memory");
+            float sc2[kFUnroll];
+#pragma unroll
+            for (int u = 0; u < kFUnroll; u += 2) {
+                const float2 v = lut2_score2(sh.u.tab.t2, rows[u], rows[u + 1], lane, qmu);
+                sc2[u] = v.x;
+                sc2[u + 1] = v.y;
+            }
 #pragma unroll
             for (int u = 0; u < kFUnroll; ++u) {
                 const int i = i0 + u;
-                const int t = t0 + kFT * i + 32 * warp + lane;
+                if (i >= npt) break;
+                const int t = t0 + kFT * i + my;
+                uint16_t e = 0;
                 if (t >= tstart && t < t1) {
-                    const float sv = lut2_score(sh.u.tab.t2, rows[u], lane, qmu);
-                    const int bi = bin_of(sv);
+                    const float sv = sc2[u];
+                    int bi = 0;
+                    if (!bin_flat) bi = min(max(__float2int_rz((sv - bin_lo) * bin_inv), 0), kFBins - 1);
                     atomicAdd(&sh.hist[bi], 1u);
-                    binpk[i >> 1] |= static_cast<uint32_t>(bi + 1) << (16 * (i & 1));
+                    e = static_cast<uint16_t>(bi + 1);
                     if (so) so[t] = sv;
                 } else if (so && t < t1) {
                     so[t] = -INFINITY;
                 }
+                sh.bins[i * kFT + tid] = e;
             }
         }
     }
-    auto bin_at = [&](int i) -> int { return static_cast<int>((binpk[i >> 1] >> (16 * (i & 1))) & 0xFFFFu) - 1; };
-    // exact score of register slot i (recomputed: same lane, same table, same bits)
-    auto score_at = [&](int i) -> float {
-        return rescore(sh.u.tab.t2, crow, t0 + kFT * i + 32 * warp + lane, lane, qmu);
-    };
     __syncthreads();
 
     // ---- 1. local k-th bin, publish the bins at or above it
-    {
-        uint32_t total;
-        {
-            uint32_t loc = 0;
-            for (int i = tid; i < kFBins; i += kFT) loc += sh.hist[i];
-            cta_excl_scan(loc, sh.wtot, &total);
+    if (k > 0) {
+        if (tid == 0) {
+            sh.sc[0] = 0;
+            sh.sc[1] = 0;
         }
-        int bc = 0;
-        if (k > 0 && total >= static_cast<uint32_t>(k)) {
-            cta_find_bin([&](int i) { return sh.hist[i]; }, kFBins, static_cast<uint32_t>(k), sh.wtot, sh.sc);
-            bc = static_cast<int>(sh.sc[0]);
-        }
-        if (k > 0) {
-            uint32_t *gh = a.ghist + static_cast<size_t>(seg) * kFBins;
-            for (int i = bc + tid; i < kFBins; i += kFT) {
-                const uint32_t v = sh.hist[i];
-                if (v) atomicAdd(gh + i, v);
-            }
+        __syncthreads();
+        cta_find_bin<kFBins / kFT>([&](int i) { return sh.hist[i]; }, static_cast<uint32_t>(k), sh.wtot, sh.sc);
+        const int bc = static_cast<int>(sh.sc[0]);    // 0 when the chunk holds fewer than k tokens
+        uint32_t *gh = a.ghist + static_cast<size_t>(seg) * kFBins;
+        for (int i = bc + tid; i < kFBins; i += kFT) {
+            const uint32_t v = sh.hist[i];
+            if (v) atomicAdd(gh + i, v);
         }
     }
     cta_arrive(&ctl->arrive1);
     cta_wait(&ctl->arrive1, a.cps, a.status);
 
-    // ---- 2. global k-th bin b*; select higher bins, list the tokens of b*
+    // ---- 2. segment k-th bin b*; count higher bins, list the tokens of b*
     int bstar = kFBins;              // nothing selected when k == 0
     uint32_t above_bstar = 0;
     if (k > 0) {
         const uint32_t *gh = a.ghist + static_cast<size_t>(seg) * kFBins;
-        cta_find_bin([&](int i) { return __ldcg(gh + i); }, kFBins, static_cast<uint32_t>(k), sh.wtot, sh.sc);
+        cta_find_bin<kFBins / kFT>([&](int i) { return __ldcg(gh + i); }, static_cast<uint32_t>(k), sh.wtot, sh.sc);
         bstar = static_cast<int>(sh.sc[0]);
         above_bstar = sh.sc[1];
-    }
-    {
         uint32_t mine = 0;
         uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
-#pragma unroll
-        for (int i = 0; i < NPT; ++i) {
-            const int t = t0 + kFT * i + 32 * warp + lane;
-            const int bi = bin_at(i);
-            if (bi < 0 || k == 0) continue;
-            if (bi > bstar) {
-                ++mine;
-            } else if (bi == bstar) {
-                const int slot = atomicAdd(&ctl->ncand, 1);
-                if (slot < a.cand_cap) cand[slot] = make_uint2(score_key(score_at(i)), static_cast<uint32_t>(t));
+        const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
+#pragma unroll 1
+        for (int row = warp; row * kFRow < a.chunk; row += kFW) {
+            const int p0 = row * kFRow + 8 * lane;
+            const uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
+            const uint32_t gt = mask8(half_gt(w.x, b2), half_gt(w.y, b2), half_gt(w.z, b2), half_gt(w.w, b2));
+            const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
+            mine += __popc(gt);
+            // selected for sure: the code and value rows are needed by the
+            // attention pass, so they go to L2 now
+            for (uint32_t mm = gt; mm; mm &= mm - 1) {
+                const int t = t0 + p0 + __ffs(mm) - 1;
+                prefetch_l2(crow + t);
+                prefetch_l2(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB);
+                if (EB * kHeadDim > 128) prefetch_l2(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB + 128);
+            }
+            // tokens of the threshold bin: exact key needed.  The lane that
+            // scored token t0 + p is p mod 32 (the table's bank rotation), so
+            // the warp hands each one to that lane.
+            uint32_t todo = __ballot_sync(0xffffffffu, eq != 0);
+            while (todo) {
+                const int src = __ffs(todo) - 1;
+                todo &= todo - 1;
+                const uint32_t em = __shfl_sync(0xffffffffu, eq, src);
+                for (uint32_t mm = em; mm; mm &= mm - 1) {
+                    const int p = row * kFRow + 8 * src + __ffs(mm) - 1;
+                    if (lane == (p & 31))
+                        emit_candidate(sh.u.tab.t2, crow, t0 + p, lane, qmu, &ctl->ncand, cand, a.cand_cap);
+                }
             }
         }
         uint32_t tot;
@@ -398,117 +474,73 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         if (tid == 0) a.selcnt[static_cast<size_t>(seg) * a.cps + c] = static_cast<int32_t>(tot);
     }
     cta_arrive(&ctl->arrive2);
-    cta_wait(&ctl->arrive2, a.cps, a.status);
 
-    // ---- 3. exact threshold among the candidates (same result in every CTA)
-    uint32_t T = 0xFFFFFFFFu, tie_idx = 0;
-    bool have_ties = false;
-    if (k > 0) {
-        const int ncand = min(__ldcg(&ctl->ncand), a.cand_cap);
-        const uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
-        const bool staged = ncand <= kFCandSmem;
-        if (staged) {
-            for (int e = tid; e < ncand; e += kFT) {
-                const uint2 v = __ldcg(cand + e);
-                sh.ckey[e] = v.x;
-                sh.cidx[e] = static_cast<int32_t>(v.y);
+    // Tokens above b* are selected whatever the candidates decide, so they
+    // (and this CTA's share of the sinks) are attended first, while the
+    // other CTAs finish the candidate list; the winners of the threshold bin
+    // follow in a second pass over the same code, continuing the same online
+    // softmax.  Entry bit 15 marks a token of the first pass, bit 14 one of
+    // the second.
+    const int nrows = (a.chunk + kFRow - 1) / kFRow;           // <= 64
+    const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
+    auto row_mask = [&](int row, uint32_t bit2) -> uint32_t {
+        const uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + row * kFRow + 8 * lane);
+        return mask8(__vcmpne2(w.x & bit2, 0u), __vcmpne2(w.y & bit2, 0u), __vcmpne2(w.z & bit2, 0u),
+                     __vcmpne2(w.w & bit2, 0u));
+    };
+    // sets bit2 on the entries picked by pick(row, words) and counts them per row;
+    // returns the total, with sh.rowcnt turned into each row's ordinal base
+    auto mark_rows = [&](uint32_t bit2, auto pick) -> uint32_t {
+#pragma unroll 1
+        for (int row = warp; row < nrows; row += kFW) {
+            const int p0 = row * kFRow + 8 * lane;
+            uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
+            const uint32_t m = pick(p0, w);
+            if (m) {
+                const uint32_t lo = bit2 & 0xFFFFu, hi = bit2 & 0xFFFF0000u;
+                w.x |= ((m & 1u) ? lo : 0u) | ((m & 2u) ? hi : 0u);
+                w.y |= ((m & 4u) ? lo : 0u) | ((m & 8u) ? hi : 0u);
+                w.z |= ((m & 16u) ? lo : 0u) | ((m & 32u) ? hi : 0u);
+                w.w |= ((m & 64u) ? lo : 0u) | ((m & 128u) ? hi : 0u);
+                *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
             }
-            __syncthreads();
-        }
-        auto ckey = [&](int e) -> uint32_t { return staged ? sh.ckey[e] : __ldcg(cand + e).x; };
-        auto cidx = [&](int e) -> uint32_t {
-            return staged ? static_cast<uint32_t>(sh.cidx[e]) : __ldcg(cand + e).y;
-        };
-        const uint32_t need = static_cast<uint32_t>(k) - above_bstar;   // >= 1
-        uint32_t ties_needed;
-        T = cta_radix_select(ckey, [&](int) { return true; }, ncand, need, sh.hist, sh.wtot, sh.sc, &ties_needed);
-        // the ties_needed lowest token indices among keys equal to T
-        uint32_t left;
-        const uint32_t inv_idx = cta_radix_select([&](int e) { return ~cidx(e); },
-                                                  [&](int e) { return ckey(e) == T; }, ncand, ties_needed,
-                                                  sh.hist, sh.wtot, sh.sc, &left);
-        tie_idx = ~inv_idx;          // ties with token index <= tie_idx are selected
-        have_ties = true;
-    }
-
-    // ---- selection bits in registers (the exact keys of threshold-bin
-    // tokens are recomputed, so the scoring tables must still be intact)
-    uint32_t selmask = 0, selmask_hi = 0;      // bit i: register slot i selected
-    {
+            uint32_t cnt = __popc(m);
 #pragma unroll
-        for (int i = 0; i < NPT; ++i) {
-            const int bi = bin_at(i);
-            bool sel = false;
-            if (bi >= 0 && k > 0) {
-                if (bi > bstar) {
-                    sel = true;
-                } else if (bi == bstar) {
-                    const uint32_t key = score_key(score_at(i));
-                    const uint32_t t = static_cast<uint32_t>(t0 + kFT * i + 32 * warp + lane);
-                    sel = key > T || (have_ties && key == T && t <= tie_idx);
-                }
-            }
-            if (sel) {
-                if (i < 32) selmask |= 1u << i;
-                else selmask_hi |= 1u << (i - 32);
-            }
-        }
-    }
-    auto sel_bit = [&](int i) -> bool { return i < 32 ? ((selmask >> i) & 1u) : ((selmask_hi >> (i - 32)) & 1u); };
-    __syncthreads();                           // scoring tables dead from here on
-
-    // ---- ordinals in ascending token order: group (i, w) holds tokens
-    // t0 + 256 i + 32 w + [0, 32), ordered by i then w
-    uint32_t *grp = sh.u.at.grp;
-#pragma unroll
-    for (int i = 0; i < NPT; ++i) {
-        const uint32_t bal = __ballot_sync(0xffffffffu, sel_bit(i));
-        if (lane == 0) grp[i * kFW + warp] = __popc(bal);
-    }
-    __syncthreads();
-    uint32_t n_sel;
-    {
-        constexpr int per = (NPT * kFW + kFT - 1) / kFT;
-        uint32_t v[per > 0 ? per : 1];
-        uint32_t loc = 0;
-#pragma unroll
-        for (int j = 0; j < per; ++j) {
-            const int gi = tid * per + j;
-            v[j] = gi < NPT * kFW ? grp[gi] : 0u;
-            loc += v[j];
-        }
-        uint32_t run = cta_excl_scan(loc, sh.wtot, &n_sel);
-#pragma unroll
-        for (int j = 0; j < per; ++j) {
-            const int gi = tid * per + j;
-            if (gi < NPT * kFW) grp[gi] = run;
-            run += v[j];
+            for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+            if (lane == 0) sh.rowcnt[row] = cnt;
         }
         __syncthreads();
-    }
+        uint32_t total;
+        const uint32_t v = tid < nrows ? sh.rowcnt[tid] : 0u;
+        const uint32_t run = cta_excl_scan(v, sh.wtot, &total);
+        if (tid < nrows) sh.rowcnt[tid] = run;
+        __syncthreads();
+        return total;
+    };
+    const uint32_t kSure = 0x80008000u, kWin = 0x40004000u;
+    const uint32_t n_sure = k > 0 ? mark_rows(kSure, [&](int, uint4 w) -> uint32_t {
+        return mask8(half_gt(w.x, b2), half_gt(w.y, b2), half_gt(w.z, b2), half_gt(w.w, b2));
+    }) : 0u;
 
-    // offset of this chunk's selection in idx_out: the selected tokens of the
-    // earlier chunks (their higher-bin counts plus their winning candidates)
-    uint32_t out_base = 0;
-    if (a.idx_out && k > 0) {
-        uint32_t before = 0;
-        for (int cc = tid; cc < c; cc += kFT)
-            before += static_cast<uint32_t>(__ldcg(a.selcnt + static_cast<size_t>(seg) * a.cps + cc));
-        const int ncand = min(__ldcg(&ctl->ncand), a.cand_cap);
-        const uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
-        for (int e = tid; e < ncand; e += kFT) {
-            const uint2 v = __ldcg(cand + e);
-            const bool win = v.x > T || (have_ties && v.x == T && v.y <= tie_idx);
-            if (win && static_cast<int>(v.y) < t0) ++before;
+    // per-head LUTs: q_h[4s:4s+4] . c[s][j] (the codebook again, from L2)
+    {
+        const float4 *cb = reinterpret_cast<const float4 *>(a.codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
+#pragma unroll 1
+        for (int r = tid; r < kSubspaces * kClusters; r += kFT) {
+            const int s = r >> 4;
+            const float4 c4 = __ldg(cb + r);
+#pragma unroll
+            for (int g = 0; g < GM; ++g) {
+                float v = sh.qs[g][4 * s] * c4.x;
+                v = fmaf(sh.qs[g][4 * s + 1], c4.y, v);
+                v = fmaf(sh.qs[g][4 * s + 2], c4.z, v);
+                v = fmaf(sh.qs[g][4 * s + 3], c4.w, v);
+                sh.u.at.luth[r][g] = v;
+            }
         }
-        cta_excl_scan(before, sh.wtot, &out_base);
     }
-
-    // ---- attention over this CTA's selected tokens and its share of the sinks
     const int n_sinks = min(a.num_sinks, n_tok);
     const int my_sinks = (n_sinks > c) ? (n_sinks - c + a.cps - 1) / a.cps : 0;   // sinks t = c (mod cps)
-    const uint32_t n_list = n_sel + static_cast<uint32_t>(my_sinks);
-    const size_t kv_seg = static_cast<size_t>(seg) * a.nmax;
     if (tid < GM) {
         sh.run_m[tid] = -INFINITY;
         sh.run_l[tid] = 0.f;
@@ -516,138 +548,249 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     float o[GM][4];
 #pragma unroll
     for (int g = 0; g < GM; ++g) o[g][0] = o[g][1] = o[g][2] = o[g][3] = 0.f;
-    int32_t *io = a.idx_out ? a.idx_out + static_cast<size_t>(seg) * a.kmax : nullptr;
-    for (uint32_t wbase = 0; wbase < n_list; wbase += kFListCap) {
-        // stage the window [wbase, wbase + kFListCap) of the ordered list
-        asm volatile("" ::: "memory");
-        const uint32_t wn = min(static_cast<uint32_t>(kFListCap), n_list - wbase);
-#pragma unroll
-        for (int i = 0; i < NPT; ++i) {
-            const uint32_t bal = __ballot_sync(0xffffffffu, sel_bit(i));
-            if (sel_bit(i)) {
-                const uint32_t ord = grp[i * kFW + warp] + __popc(bal & ((1u << lane) - 1u));
-                const int t = t0 + kFT * i + 32 * warp + lane;
-                if (ord >= wbase && ord < wbase + kFListCap) sh.u.at.list[ord - wbase] = t;
-                if (io && wbase == 0 && out_base + ord < static_cast<uint32_t>(k)) io[out_base + ord] = t;
+    uint32_t win_before = 0;           // this thread's share of winners with token < t0
+    uint32_t n_win = 0;
+
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        uint32_t n_sel = n_sure, bit2 = kSure, n_list = n_sure + static_cast<uint32_t>(my_sinks);
+        if (pass == 1) {
+            // ---- exact winners among the threshold-bin candidates (the same
+            // answer in every CTA): a candidate wins when fewer than `need`
+            // candidates come before it (key descending, token ascending)
+            cta_wait(&ctl->arrive2, a.cps, a.status);
+            for (int i = tid; i < kFMaxChunk / 32; i += kFT) sh.u.sel.winbits[i] = 0;
+            __syncthreads();
+            if (k > 0) {
+                const int ncand = min(__ldcg(&ctl->ncand), a.cand_cap);
+                const uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
+                const uint32_t need = static_cast<uint32_t>(k) - above_bstar;   // >= 1
+                if (ncand <= kFRankMax) {
+                    for (int e = tid; e < ncand; e += kFT) {
+                        const uint2 v = __ldcg(cand + e);
+                        sh.u.sel.ckey[e] = v.x;
+                        sh.u.sel.cidx[e] = static_cast<int32_t>(v.y);
+                    }
+                    __syncthreads();
+                    for (int e = tid; e < ncand; e += kFT) {
+                        const uint32_t ke = sh.u.sel.ckey[e], ie = static_cast<uint32_t>(sh.u.sel.cidx[e]);
+                        uint32_t rank = 0;
+                        for (int f = 0; f < ncand; ++f) {
+                            const uint32_t kf = sh.u.sel.ckey[f];
+                            rank += (kf > ke) || (kf == ke && static_cast<uint32_t>(sh.u.sel.cidx[f]) < ie);
+                        }
+                        if (rank < need) {
+                            const int rel = static_cast<int>(ie) - t0;
+                            if (rel >= 0 && rel < a.chunk) atomicOr(&sh.u.sel.winbits[rel >> 5], 1u << (rel & 31));
+                            else if (rel < 0) ++win_before;
+                        }
+                    }
+                } else {
+                    win_before += refine_by_radix(cand, ncand, need, t0, a.chunk, sh.u.sel.winbits, sh.hist, sh.wtot,
+                                                  sh.sc);
+                }
+                __syncthreads();
+                n_win = mark_rows(kWin, [&](int p0, uint4 w) -> uint32_t {
+                    const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
+                    return eq ? (eq & ((sh.u.sel.winbits[p0 >> 5] >> (p0 & 31)) & 0xFFu)) : 0u;
+                });
             }
+            n_sel = n_win;
+            bit2 = kWin;
+            n_list = n_win;
         }
-        for (uint32_t e = tid; e < wn; e += kFT) {
-            const uint32_t ord = wbase + e;
-            if (ord >= n_sel) sh.u.at.list[e] = -1 - static_cast<int32_t>(c + (ord - n_sel) * a.cps);   // a sink
-        }
-        __syncthreads();
-        for (uint32_t tbase = 0; tbase < wn; tbase += kFTile) {
-            const uint32_t tile_n = min(static_cast<uint32_t>(kFTile), wn - tbase);
-            // logits, one list entry per thread
-            {
-                float lg[GM];
+#pragma unroll 1
+        for (uint32_t wbase = 0; wbase < n_list; wbase += kFListCap) {
+            // stage the window [wbase, wbase + kFListCap) of this pass's list:
+            // selected tokens in ascending order, then (first pass) the sinks
+            const uint32_t wn = min(static_cast<uint32_t>(kFListCap), n_list - wbase);
+#pragma unroll 1
+            for (int row = warp; row < nrows; row += kFW) {
+                const uint32_t m = row_mask(row, bit2);
+                uint32_t incl = __popc(m);
 #pragma unroll
-                for (int g = 0; g < GM; ++g) lg[g] = -INFINITY;
-                if (static_cast<uint32_t>(tid) < tile_n) {
-                    const int32_t ent = sh.u.at.list[tbase + tid];
-                    if (ent >= 0) {
-                        const uint4 row = __ldg(reinterpret_cast<const uint4 *>(a.codes) + kv_seg + ent);
-                        const uint32_t w[4] = {row.x, row.y, row.z, row.w};
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += o2;
+                }
+                uint32_t ord = sh.rowcnt[row] + incl - __popc(m);
+                for (uint32_t mm = m; mm; mm &= mm - 1, ++ord) {
+                    const int t = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
+                    if (ord >= wbase && ord < wbase + kFListCap) sh.u.at.list[ord - wbase] = t;
+                }
+            }
+            for (uint32_t e = tid; e < wn; e += kFT) {
+                const uint32_t ord = wbase + e;
+                if (ord >= n_sel) sh.u.at.list[e] = -1 - static_cast<int32_t>(c + (ord - n_sel) * a.cps);   // a sink
+            }
+            __syncthreads();
+#pragma unroll 1
+            for (uint32_t tbase = 0; tbase < wn; tbase += kFTile) {
+                const uint32_t tile_n = min(static_cast<uint32_t>(kFTile), wn - tbase);
+                // logits, one list entry per thread
+                {
+                    float lg[GM];
+#pragma unroll
+                    for (int g = 0; g < GM; ++g) lg[g] = -INFINITY;
+                    if (static_cast<uint32_t>(tid) < tile_n) {
+                        const int32_t ent = sh.u.at.list[tbase + tid];
                         float acc[GM];
 #pragma unroll
                         for (int g = 0; g < GM; ++g) acc[g] = 0.f;
+                        if (ent >= 0) {
+                            const uint4 row = __ldg(crow + ent);
+                            const uint32_t w[4] = {row.x, row.y, row.z, row.w};
+#pragma unroll 8
+                            for (int s = 0; s < kSubspaces; ++s) {
+                                const int j = (w[s >> 3] >> (4 * (s & 7))) & 15;
+                                const float *lp = sh.u.at.luth[s * kClusters + j];
 #pragma unroll
-                        for (int s = 0; s < kSubspaces; ++s) {
-                            const int j = (w[s >> 3] >> (4 * (s & 7))) & 15;
-                            const float *lp = sh.luth[s * kClusters + j];
-#pragma unroll
-                            for (int g = 0; g < GM; g += 4) {
-                                const float4 v4 = *reinterpret_cast<const float4 *>(lp + g);
-                                acc[g] += v4.x;
-                                acc[g + 1] += v4.y;
-                                acc[g + 2] += v4.z;
-                                acc[g + 3] += v4.w;
+                                for (int g = 0; g < GM; g += 4) {
+                                    const float4 v4 = *reinterpret_cast<const float4 *>(lp + g);
+                                    acc[g] += v4.x;
+                                    acc[g + 1] += v4.y;
+                                    acc[g + 2] += v4.z;
+                                    acc[g + 3] += v4.w;
+                                }
                             }
-                        }
 #pragma unroll
-                        for (int g = 0; g < GM; ++g) lg[g] = (acc[g] + sh.qmu_h[g]) * a.scale;
-                    } else {
-                        const int t = -1 - ent;
-                        const char *krow = static_cast<const char *>(a.K) + (kv_seg + t) * kHeadDim * EB;
-                        float acc[GM];
+                            for (int g = 0; g < GM; ++g) lg[g] = (acc[g] + sh.qmu_h[g]) * a.scale;
+                        } else {
+                            const char *krow = static_cast<const char *>(a.K) + (kv_seg + (-1 - ent)) * kHeadDim * EB;
+#pragma unroll 2
+                            for (int d = 0; d < kHeadDim; d += 4) {
+                                const float4 kv = load4<DT>(krow, d);
 #pragma unroll
-                        for (int g = 0; g < GM; ++g) acc[g] = 0.f;
-                        for (int d = 0; d < kHeadDim; d += 4) {
-                            const float4 kv = load4<DT>(krow, d);
-#pragma unroll
-                            for (int g = 0; g < GM; ++g) {
-                                acc[g] = fmaf(sh.qs[g][d], kv.x, acc[g]);
-                                acc[g] = fmaf(sh.qs[g][d + 1], kv.y, acc[g]);
-                                acc[g] = fmaf(sh.qs[g][d + 2], kv.z, acc[g]);
-                                acc[g] = fmaf(sh.qs[g][d + 3], kv.w, acc[g]);
+                                for (int g = 0; g < GM; ++g) {
+                                    acc[g] = fmaf(sh.qs[g][d], kv.x, acc[g]);
+                                    acc[g] = fmaf(sh.qs[g][d + 1], kv.y, acc[g]);
+                                    acc[g] = fmaf(sh.qs[g][d + 2], kv.z, acc[g]);
+                                    acc[g] = fmaf(sh.qs[g][d + 3], kv.w, acc[g]);
+                                }
                             }
-                        }
 #pragma unroll
-                        for (int g = 0; g < GM; ++g) lg[g] = acc[g] * a.scale;
+                            for (int g = 0; g < GM; ++g) lg[g] = acc[g] * a.scale;
+                        }
+                    }
+#pragma unroll
+                    for (int g = 0; g < GM; ++g) {
+                        const float v = (g < group) ? lg[g] : -INFINITY;
+                        sh.u.at.logit[g][tid] = v;
+                        float mx = v;
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                        if (lane == 0) sh.tile_stat[warp][g] = mx;
                     }
                 }
+                __syncthreads();
+                // new running max per head and the rescale factor of what came before
+                float alpha[GM], mnew[GM];
 #pragma unroll
                 for (int g = 0; g < GM; ++g) {
-                    const float v = (g < group) ? lg[g] : -INFINITY;
-                    sh.u.at.logit[g][tid] = v;
-                    float mx = v;
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                    if (lane == 0) sh.tile_stat[warp][g] = mx;
+                    float mx = sh.run_m[g];
+                    for (int w = 0; w < kFW; ++w) mx = fmaxf(mx, sh.tile_stat[w][g]);
+                    mnew[g] = mx;
+                    alpha[g] = (sh.run_m[g] == -INFINITY) ? 0.f : __expf(sh.run_m[g] - mx);
                 }
-            }
-            __syncthreads();
-            // new running max per head and the rescale factor of what came before
-            float alpha[GM], mnew[GM];
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                float mx = sh.run_m[g];
-                for (int w = 0; w < kFW; ++w) mx = fmaxf(mx, sh.tile_stat[w][g]);
-                mnew[g] = mx;
-                alpha[g] = (sh.run_m[g] == -INFINITY) ? 0.f : expf(sh.run_m[g] - mx);
-            }
-            __syncthreads();
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                const float lv = sh.u.at.logit[g][tid];
-                const float pr = (lv == -INFINITY) ? 0.f : expf(lv - mnew[g]);
-                sh.u.at.logit[g][tid] = pr;
-                float sm = pr;
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
-                if (lane == 0) sh.tile_stat[warp][g] = sm;
-            }
-            __syncthreads();
-            if (tid < GM) {
-                float sm = 0.f;
-                for (int w = 0; w < kFW; ++w) sm += sh.tile_stat[w][tid];
-                sh.run_l[tid] = sh.run_l[tid] * alpha[tid] + sm;
-                sh.run_m[tid] = mnew[tid];
-            }
-            // o = alpha o + sum_e p_e V[t_e]; warp w takes entries w, w + 8, ...
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                o[g][0] *= alpha[g];
-                o[g][1] *= alpha[g];
-                o[g][2] *= alpha[g];
-                o[g][3] *= alpha[g];
-            }
-            for (uint32_t e = warp; e < tile_n; e += kFW) {
-                const int32_t ent = sh.u.at.list[tbase + e];
-                const int t = ent >= 0 ? ent : -1 - ent;
-                const float4 v = load4<DT>(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB, lane * 4);
+                __syncthreads();
 #pragma unroll
                 for (int g = 0; g < GM; ++g) {
-                    const float pr = sh.u.at.logit[g][e];
-                    o[g][0] = fmaf(pr, v.x, o[g][0]);
-                    o[g][1] = fmaf(pr, v.y, o[g][1]);
-                    o[g][2] = fmaf(pr, v.z, o[g][2]);
-                    o[g][3] = fmaf(pr, v.w, o[g][3]);
+                    const float lv = sh.u.at.logit[g][tid];
+                    const float pr = (lv == -INFINITY) ? 0.f : __expf(lv - mnew[g]);
+                    sh.u.at.logit[g][tid] = pr;
+                    float sm = pr;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+                    if (lane == 0) sh.tile_stat[warp][g] = sm;
                 }
+                __syncthreads();
+                if (tid < GM) {
+                    float sm = 0.f;
+                    for (int w = 0; w < kFW; ++w) sm += sh.tile_stat[w][tid];
+                    sh.run_l[tid] = sh.run_l[tid] * alpha[tid] + sm;
+                    sh.run_m[tid] = mnew[tid];
+                }
+                // o = alpha o + sum_e p_e V[t_e]; warp w takes entries w, w + 8, ...
+#pragma unroll
+                for (int g = 0; g < GM; ++g) {
+                    o[g][0] *= alpha[g];
+                    o[g][1] *= alpha[g];
+                    o[g][2] *= alpha[g];
+                    o[g][3] *= alpha[g];
+                }
+#pragma unroll 1
+                for (uint32_t e0 = warp; e0 < tile_n; e0 += kFVRows * kFW) {
+                    float4 v[kFVRows];
+#pragma unroll
+                    for (int u = 0; u < kFVRows; ++u) {
+                        const uint32_t e = e0 + u * kFW;
+                        if (e < tile_n) {
+                            const int32_t ent = sh.u.at.list[tbase + e];
+                            const int t = ent >= 0 ? ent : -1 - ent;
+                            v[u] = load4<DT>(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB, lane * 4);
+                        } else {
+                            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kFVRows; ++u) {
+                        const uint32_t e = e0 + u * kFW;
+                        const float4 vv = v[u];
+#pragma unroll
+                        for (int g = 0; g < GM; ++g) {
+                            const float pr = e < tile_n ? sh.u.at.logit[g][e] : 0.f;
+                            o[g][0] = fmaf(pr, vv.x, o[g][0]);
+                            o[g][1] = fmaf(pr, vv.y, o[g][1]);
+                            o[g][2] = fmaf(pr, vv.z, o[g][2]);
+                            o[g][3] = fmaf(pr, vv.w, o[g][3]);
+                        }
+                    }
+                }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
+
+    // selected tokens in ascending order into idx_out, after the selected
+    // tokens of the earlier chunks (their higher-bin counts plus their winners)
+    if (a.idx_out && k > 0) {
+        uint32_t before = win_before;
+        for (int cc = tid; cc < c; cc += kFT)
+            before += static_cast<uint32_t>(__ldcg(a.selcnt + static_cast<size_t>(seg) * a.cps + cc));
+        uint32_t out_base;
+        cta_excl_scan(before, sh.wtot, &out_base);
+#pragma unroll 1
+        for (int row = warp; row < nrows; row += kFW) {
+            const uint32_t m = row_mask(row, kSure | kWin);
+            uint32_t cnt = __popc(m);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+            if (lane == 0) sh.rowcnt[row] = cnt;
+        }
+        __syncthreads();
+        {
+            uint32_t total;
+            const uint32_t v = tid < nrows ? sh.rowcnt[tid] : 0u;
+            const uint32_t run = cta_excl_scan(v, sh.wtot, &total);
+            if (tid < nrows) sh.rowcnt[tid] = run;
+            __syncthreads();
+        }
+        int32_t *io = a.idx_out + static_cast<size_t>(seg) * a.kmax;
+#pragma unroll 1
+        for (int row = warp; row < nrows; row += kFW) {
+            const uint32_t m = row_mask(row, kSure | kWin);
+            uint32_t incl = __popc(m);
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o2;
+            }
+            uint32_t ord = out_base + sh.rowcnt[row] + incl - __popc(m);
+            for (uint32_t mm = m; mm; mm &= mm - 1, ++ord)
+                if (ord < static_cast<uint32_t>(k)) io[ord] = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
+        }
+    }
+
     // reduce o over the warps and write this CTA's partial
 #pragma unroll
     for (int g = 0; g < GM; ++g)
@@ -671,6 +814,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     __syncthreads();
     if (!sh.last) return;
     __threadfence();
+#pragma unroll 1
     for (int e = tid; e < group * kHeadDim; e += kFT) {
         const int g = e / kHeadDim, d = e % kHeadDim;
         float mx = -INFINITY;
@@ -681,12 +825,12 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
             for (int cc = 0; cc < a.cps; ++cc) {
                 const size_t pb = (static_cast<size_t>(seg) * a.cps + cc) * GM + g;
                 const float2 ml = __ldcg(a.part_ml + pb);
-                const float wgt = (ml.x == -INFINITY) ? 0.f : expf(ml.x - mx);
+                const float wgt = (ml.x == -INFINITY) ? 0.f : __expf(ml.x - mx);
                 l = fmaf(ml.y, wgt, l);
                 acc = fmaf(__ldcg(a.part_o + pb * kHeadDim + d), wgt, acc);
             }
         }
-        const float r = (l > 0.f) ? acc / l : 0.f;
+        const float r = (l > 0.f) ? __fdividef(acc, l) : 0.f;
         const size_t orow = (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group + g) * kHeadDim + d;
         if (DT == SIKV_DTYPE_F32)
             static_cast<float *>(a.out)[orow] = r;
@@ -707,9 +851,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     }
 }
 
-template <int DT, int GM, int NPT>
-sikv_status launch_fused_t(const sikv_params &p, const FusedArgs &args, const FusedPlan &plan, cudaStream_t stream) {
-    auto kern = decode_fused_kernel<DT, GM, NPT>;
+template <int DT, int GM>
+sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStream_t stream) {
+    auto kern = decode_fused_kernel<DT, GM>;
     const size_t smem = sizeof(FusedSmem<GM>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SIKV_ERR_CUDA;
@@ -717,26 +861,14 @@ sikv_status launch_fused_t(const sikv_params &p, const FusedArgs &args, const Fu
     void *params[] = {&a};
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(plan.grid),
                                                       dim3(kFT), params, smem, stream);
-    (void)p;
     return e == cudaSuccess ? SIKV_OK : SIKV_ERR_CUDA;
 }
 
 template <int DT, int GM>
-sikv_status dispatch_npt(const sikv_params &p, const FusedArgs &args, const FusedPlan &plan, cudaStream_t stream) {
-    switch (plan.npt) {
-        case 8: return launch_fused_t<DT, GM, 8>(p, args, plan, stream);
-        case 16: return launch_fused_t<DT, GM, 16>(p, args, plan, stream);
-        case 32: return launch_fused_t<DT, GM, 32>(p, args, plan, stream);
-        case 64: return launch_fused_t<DT, GM, 64>(p, args, plan, stream);
-        default: return SIKV_ERR_UNSUPPORTED;
-    }
-}
-
-template <int DT, int GM, int NPT>
 int occupancy_of() {
     // the occupancy calculator honours the kernel's dynamic shared-memory
     // limit, which must be raised above the 48 KB default first
-    auto kern = decode_fused_kernel<DT, GM, NPT>;
+    auto kern = decode_fused_kernel<DT, GM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FusedSmem<GM>)) !=
         cudaSuccess)
         return 0;
@@ -744,17 +876,6 @@ int occupancy_of() {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kFT, sizeof(FusedSmem<GM>)) != cudaSuccess)
         return 0;
     return blocks;
-}
-
-template <int DT, int GM>
-int occupancy_npt(int npt) {
-    switch (npt) {
-        case 8: return occupancy_of<DT, GM, 8>();
-        case 16: return occupancy_of<DT, GM, 16>();
-        case 32: return occupancy_of<DT, GM, 32>();
-        case 64: return occupancy_of<DT, GM, 64>();
-        default: return 0;
-    }
 }
 
 }  // namespace
@@ -789,9 +910,13 @@ FusedPlan fused_plan(const sikv_params &p) {
     const int segs = p.batch * p.num_kv_heads;
     const int sms = device_sm_count();
     if (sms <= 0) return plan;
-    // two CTAs per SM is the design point; confirm with the occupancy calculator
-    const int per_sm_guess = 2;
-    int cps = (sms * per_sm_guess) / segs;
+    int occ = 0;
+    if (p.dtype == SIKV_DTYPE_BF16)
+        occ = gm == 4 ? occupancy_of<SIKV_DTYPE_BF16, 4>() : occupancy_of<SIKV_DTYPE_BF16, 8>();
+    else
+        occ = gm == 4 ? occupancy_of<SIKV_DTYPE_F32, 4>() : occupancy_of<SIKV_DTYPE_F32, 8>();
+    if (occ < 1) return plan;
+    int cps = (sms * occ) / segs;
     const int min_chunk = 2048;
     cps = std::min(cps, (p.max_seq_len + min_chunk - 1) / min_chunk);
     cps = std::min(cps, kFusedMaxCps);
@@ -799,20 +924,11 @@ FusedPlan fused_plan(const sikv_params &p) {
     int chunk = (p.max_seq_len + cps - 1) / cps;
     chunk = (chunk + kFT - 1) / kFT * kFT;
     cps = (p.max_seq_len + chunk - 1) / chunk;
-    const int npt_need = chunk / kFT;
-    int npt = 8;
-    while (npt < npt_need) npt *= 2;
-    if (npt > 64) return plan;
-    int occ = 0;
-    if (p.dtype == SIKV_DTYPE_BF16)
-        occ = gm == 4 ? occupancy_npt<SIKV_DTYPE_BF16, 4>(npt) : occupancy_npt<SIKV_DTYPE_BF16, 8>(npt);
-    else
-        occ = gm == 4 ? occupancy_npt<SIKV_DTYPE_F32, 4>(npt) : occupancy_npt<SIKV_DTYPE_F32, 8>(npt);
-    if (occ < 1 || static_cast<long long>(segs) * cps > static_cast<long long>(occ) * sms) return plan;
+    if (chunk > kFMaxChunk) return plan;
     plan.ok = true;
     plan.cps = cps;
     plan.chunk = chunk;
-    plan.npt = npt;
+    plan.npt = chunk / kFT;
     plan.gm = gm;
     plan.grid = segs * cps;
     return plan;
@@ -842,6 +958,7 @@ sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, con
     a.kmax = p.max_topk;
     a.cps = plan.cps;
     a.chunk = plan.chunk;
+    a.npt = plan.npt;
     a.cand_cap = static_cast<int>(fused_cand_cap(p));
     a.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf(static_cast<float>(p.head_dim));
     a.ghist = reinterpret_cast<uint32_t *>(ws + L.ghist);
@@ -852,10 +969,10 @@ sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, con
     a.part_ml = reinterpret_cast<float2 *>(ws + L.part_ml);
     a.status = status;
     if (p.dtype == SIKV_DTYPE_BF16)
-        return plan.gm == 4 ? dispatch_npt<SIKV_DTYPE_BF16, 4>(p, a, plan, stream)
-                            : dispatch_npt<SIKV_DTYPE_BF16, 8>(p, a, plan, stream);
-    return plan.gm == 4 ? dispatch_npt<SIKV_DTYPE_F32, 4>(p, a, plan, stream)
-                        : dispatch_npt<SIKV_DTYPE_F32, 8>(p, a, plan, stream);
+        return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_BF16, 4>(a, plan, stream)
+                            : launch_fused_t<SIKV_DTYPE_BF16, 8>(a, plan, stream);
+    return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_F32, 4>(a, plan, stream)
+                        : launch_fused_t<SIKV_DTYPE_F32, 8>(a, plan, stream);
 }
 
 }  // namespace sikv

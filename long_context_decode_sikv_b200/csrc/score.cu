@@ -24,13 +24,20 @@ score_kernel(const void *__restrict__ q, const uint8_t *__restrict__ codes,
              float *__restrict__ scores, int32_t *status) {
     extern __shared__ __align__(16) unsigned char score_smem[];
     ScoreTables &sh = *reinterpret_cast<ScoreTables *>(score_smem);
+    // staged table inputs live in the byte table's space: they are last read
+    // before the barrier that precedes the table's first write
+    float4 *cbs = reinterpret_cast<float4 *>(sh.t2);                       // 2048 floats
+    float *qs = sh.t2 + kSubspaces * kClusters * 4;                          // <= 8 x 128 floats
+    float *mus = qs + kMaxGroup * kHeadDim;                                  // 128 floats
     const int seg = blockIdx.y, b = seg / hkv, h = seg % hkv, group = hq / hkv;
     const int n_tok = load_seq_len(seq_lens, b, nmax, status);
     if (n_tok < 0) return;
     const int t_begin = blockIdx.x * kScoreChunk;
     if (t_begin >= n_tok) return;
     const int t_end = min(t_begin + kScoreChunk, n_tok);
-    build_score_tables<DT>(sh, q, codebook, mu, b, h, hq, group, seg);
+    stage_table_inputs<DT>(qs, cbs, mus, q, codebook, mu, b, h, hq, group, seg);
+    __syncthreads();
+    build_score_tables(sh, qs, cbs, mus, group);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float qmu = sh.qmu;
@@ -45,9 +52,11 @@ score_kernel(const void *__restrict__ q, const uint8_t *__restrict__ codes,
             rows[u] = (t >= num_sinks && t < t_end) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int u = 0; u < kScoreUnroll; ++u) {
-            const int t = g0 + u * kStride + lane;
-            if (t < t_end) srow[t] = (t >= num_sinks) ? lut2_score(sh.t2, rows[u], lane, qmu) : -INFINITY;
+        for (int u = 0; u < kScoreUnroll; u += 2) {
+            const float2 v = lut2_score2(sh.t2, rows[u], rows[u + 1], lane, qmu);
+            const int ta = g0 + u * kStride + lane, tb = ta + kStride;
+            if (ta < t_end) srow[ta] = (ta >= num_sinks) ? v.x : -INFINITY;
+            if (tb < t_end) srow[tb] = (tb >= num_sinks) ? v.y : -INFINITY;
         }
     }
 }

@@ -35,27 +35,43 @@ struct ScoreTables {
     float pad[3];
 };
 
-// Builds q_bar, LUT, q_bar.mu and T2 for segment (b, h) with the whole CTA.
-// Ends with a __syncthreads().
+// Loads the inputs of the tables of segment (b, h) into shared memory with one
+// round trip: the group's query rows (as fp32, `qs`, `group` x 128), the
+// segment's codebook (`cbs`, 512 float4) and channel means (`mus`, 128).
+constexpr int kTableThreads = 256;      // CTA size of every kernel that builds the tables
+
 template <int DT>
-__device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *__restrict__ q,
-                                                   const float *__restrict__ codebook,
-                                                   const float *__restrict__ mu, int b, int h,
-                                                   int hq, int group, int seg) {
+__device__ __forceinline__ void stage_table_inputs(float *qs, float4 *cbs, float *mus, const void *__restrict__ q,
+                                                   const float *__restrict__ codebook, const float *__restrict__ mu,
+                                                   int b, int h, int hq, int group, int seg) {
     constexpr int EB = ElemBytes<DT>::value;
-    const int tid = threadIdx.x, nt = blockDim.x;
+    constexpr int nt = kTableThreads;
+    const int tid = threadIdx.x;
     const char *qrow = static_cast<const char *>(q) +
                        (static_cast<size_t>(b) * hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
+#pragma unroll 1
+    for (int e = tid; e < group * kHeadDim; e += nt) qs[e] = load1<DT>(qrow, e);
+    const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
+    for (int e = tid; e < kSubspaces * kClusters; e += nt) cbs[e] = __ldg(cb + e);
+    for (int e = tid; e < kHeadDim; e += nt) mus[e] = __ldg(mu + static_cast<size_t>(seg) * kHeadDim + e);
+}
+
+// Builds q_bar, LUT, q_bar.mu and T2 from staged inputs with the whole CTA.
+// Expects the staged inputs to be visible (a __syncthreads() after staging);
+// ends with a __syncthreads().
+__device__ __forceinline__ void build_score_tables(ScoreTables &sh, const float *qs, const float4 *cbs,
+                                                   const float *mus, int group) {
+    constexpr int nt = kTableThreads;
+    const int tid = threadIdx.x;
     for (int c = tid; c < kHeadDim; c += nt) {
-        float acc = load1<DT>(qrow, c);
-        for (int g = 1; g < group; ++g) acc += load1<DT>(qrow + static_cast<size_t>(g) * kHeadDim * EB, c);
+        float acc = qs[c];
+        for (int g = 1; g < group; ++g) acc += qs[g * kHeadDim + c];
         sh.qbar[c] = acc;
     }
     __syncthreads();
-    const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
     for (int e = tid; e < kSubspaces * kClusters; e += nt) {
         const int j = e >> 5, s = e & 31;
-        const float4 c4 = __ldg(cb + s * kClusters + j);
+        const float4 c4 = cbs[s * kClusters + j];
         float v = sh.qbar[4 * s] * c4.x;
         v = fmaf(sh.qbar[4 * s + 1], c4.y, v);
         v = fmaf(sh.qbar[4 * s + 2], c4.z, v);
@@ -63,11 +79,10 @@ __device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *
         sh.lutT[e] = v;
     }
     if (tid < 32) {
-        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mu + static_cast<size_t>(seg) * kHeadDim) + tid);
-        double a = static_cast<double>(sh.qbar[4 * tid]) * m4.x;
-        a = fma(static_cast<double>(sh.qbar[4 * tid + 1]), static_cast<double>(m4.y), a);
-        a = fma(static_cast<double>(sh.qbar[4 * tid + 2]), static_cast<double>(m4.z), a);
-        a = fma(static_cast<double>(sh.qbar[4 * tid + 3]), static_cast<double>(m4.w), a);
+        double a = static_cast<double>(sh.qbar[4 * tid]) * mus[4 * tid];
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 1]), static_cast<double>(mus[4 * tid + 1]), a);
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 2]), static_cast<double>(mus[4 * tid + 2]), a);
+        a = fma(static_cast<double>(sh.qbar[4 * tid + 3]), static_cast<double>(mus[4 * tid + 3]), a);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
         if (tid == 0) sh.qmu = static_cast<float>(a);
@@ -78,6 +93,7 @@ __device__ __forceinline__ void build_score_tables(ScoreTables &sh, const void *
     // word m + 16 copy (32 distinct banks), then lanes 0..15 store word m + 32.
     {
         const int lane = tid & 31, m = lane & 15, copy = lane >> 4;
+#pragma unroll 2
         for (int byte = tid >> 5; byte < 256; byte += nt >> 5) {
             const float v = sh.lutT[(byte & 15) * kSubspaces + 2 * m] + sh.lutT[(byte >> 4) * kSubspaces + 2 * m + 1];
             float *row = sh.t2 + byte * kT2RowWords;
@@ -134,6 +150,81 @@ __device__ __forceinline__ float lut2_score(const float *__restrict__ t2, uint4 
     c += SIKV_LK(w3, 15);
 #undef SIKV_LK
     return (a + c) + qmu;
+}
+
+// Scores of two tokens computed by `lane` with their instructions interleaved
+// (four independent addition chains).  Each result is bit-identical to
+// lut2_score on the same row: same rotation, same order of additions.
+__device__ __forceinline__ float2 lut2_score2(const float *__restrict__ t2, uint4 ra, uint4 rb, int lane, float qmu) {
+    const int r = lane & 15;
+    uint32_t a0 = ra.x, a1 = ra.y, a2 = ra.z, a3 = ra.w;
+    uint32_t b0 = rb.x, b1 = rb.y, b2 = rb.z, b3 = rb.w;
+    if (r & 4) {
+        uint32_t t = a0;
+        a0 = a1;
+        a1 = a2;
+        a2 = a3;
+        a3 = t;
+        t = b0;
+        b0 = b1;
+        b1 = b2;
+        b2 = b3;
+        b3 = t;
+    }
+    if (r & 8) {
+        uint32_t t = a0;
+        a0 = a2;
+        a2 = t;
+        t = a1;
+        a1 = a3;
+        a3 = t;
+        t = b0;
+        b0 = b2;
+        b2 = t;
+        t = b1;
+        b1 = b3;
+        b3 = t;
+    }
+    const uint32_t rb3 = static_cast<uint32_t>(r & 3);
+    const uint32_t sel = rb3 * 0x1111u + 0x3210u;
+    const uint32_t x0 = __byte_perm(a0, a1, sel), x1 = __byte_perm(a1, a2, sel);
+    const uint32_t x2 = __byte_perm(a2, a3, sel), x3 = __byte_perm(a3, a0, sel);
+    const uint32_t y0 = __byte_perm(b0, b1, sel), y1 = __byte_perm(b1, b2, sel);
+    const uint32_t y2 = __byte_perm(b2, b3, sel), y3 = __byte_perm(b3, b0, sel);
+    const uint32_t base = 4u * static_cast<uint32_t>(lane);
+    const char *tb = reinterpret_cast<const char *>(t2);
+#define SIKV_LK(W, I) (*reinterpret_cast<const float *>(tb + __byte_perm((W), base, 0x6504u | (((I) & 3u) << 4)) + 4 * (I)))
+    float pa = SIKV_LK(x0, 0), qa = SIKV_LK(x2, 8), pb = SIKV_LK(y0, 0), qb = SIKV_LK(y2, 8);
+    pa += SIKV_LK(x0, 1);
+    qa += SIKV_LK(x2, 9);
+    pb += SIKV_LK(y0, 1);
+    qb += SIKV_LK(y2, 9);
+    pa += SIKV_LK(x0, 2);
+    qa += SIKV_LK(x2, 10);
+    pb += SIKV_LK(y0, 2);
+    qb += SIKV_LK(y2, 10);
+    pa += SIKV_LK(x0, 3);
+    qa += SIKV_LK(x2, 11);
+    pb += SIKV_LK(y0, 3);
+    qb += SIKV_LK(y2, 11);
+    pa += SIKV_LK(x1, 4);
+    qa += SIKV_LK(x3, 12);
+    pb += SIKV_LK(y1, 4);
+    qb += SIKV_LK(y3, 12);
+    pa += SIKV_LK(x1, 5);
+    qa += SIKV_LK(x3, 13);
+    pb += SIKV_LK(y1, 5);
+    qb += SIKV_LK(y3, 13);
+    pa += SIKV_LK(x1, 6);
+    qa += SIKV_LK(x3, 14);
+    pb += SIKV_LK(y1, 6);
+    qb += SIKV_LK(y3, 14);
+    pa += SIKV_LK(x1, 7);
+    qa += SIKV_LK(x3, 15);
+    pb += SIKV_LK(y1, 7);
+    qb += SIKV_LK(y3, 15);
+#undef SIKV_LK
+    return make_float2((pa + qa) + qmu, (pb + qb) + qmu);
 }
 
 }  // namespace sikv
