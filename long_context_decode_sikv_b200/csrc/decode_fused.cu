@@ -42,7 +42,6 @@ namespace {
 constexpr int kFT = 256;                 // threads per CTA
 constexpr int kFW = kFT / 32;            // warps per CTA
 constexpr int kFBins = 1024;             // histogram bins per segment
-constexpr int kFTile = 256;              // list entries attended per pass
 constexpr int kFListCap = 2048;          // attended tokens staged per window
 constexpr int kFMaxNpt = 64;             // token slots per thread at most
 constexpr int kFMaxChunk = kFMaxNpt * kFT;
@@ -50,8 +49,11 @@ constexpr int kFCandSmem = 1024;         // candidates staged in shared memory
 constexpr int kFRankMax = 512;           // up to this many candidates: rank directly
 constexpr int kFUnroll = 8;              // code rows in flight per thread
 constexpr int kFPrefetchRows = 16;       // code rows per thread kept ahead in L2
-constexpr int kFVRows = 8;               // value rows in flight per warp
-constexpr int kSpinLimit = 1 << 23;      // ~1 s of __nanosleep(128) polls
+constexpr int kFPend = kFBins / 4;       // threshold-bin tokens of a CTA re-scored together
+constexpr int kFDirect = kFBins / 2;     // attended tokens listed directly during the scans
+constexpr int kFWarpList = kFDirect / kFW;   // of which each warp lists (and attends) at most this many
+constexpr int kFVBytes = 4096;           // value rows staged per warp: 16 bf16 or 8 fp32 rows
+constexpr int kSpinLimit = 1 << 23;      // polls of a wait: seconds, far above any real wait
 constexpr int kFRow = 256;               // tokens per row scan of a warp (32 lanes x 8)
 
 struct FusedArgs {
@@ -87,24 +89,31 @@ struct FusedSmem {
         } sel;
         struct {
             int32_t list[kFListCap];
-            alignas(16) float logit[GM][kFTile];
-            alignas(16) float red[kFW][GM][kHeadDim];
+            union {
+                alignas(16) float red[kFW][GM][kHeadDim];     // the warps' outputs at the end
+                alignas(16) char vbuf[kFW][kFVBytes];         // each warp's staged value rows
+            };
             alignas(16) float luth[kSubspaces * kClusters][GM];   // per-head LUT, [s*16+j][g]
+            int32_t tok[kFW][32];                                 // each warp's batch tokens
         } at;
     } u;
     alignas(16) float qs[GM][kHeadDim];
     alignas(16) float mus[kHeadDim];
     alignas(16) float qmu_h[GM];
-    alignas(16) float run_m[GM];
-    alignas(16) float run_l[GM];
-    alignas(16) float tile_stat[kFW][GM];
+    alignas(16) float wm[kFW][GM];            // per-warp softmax state at the end
+    alignas(16) float wl[kFW][GM];
+    // the scoring histogram; from phase 2 on the threshold-bin tokens (offsets
+    // in [0, kFPend), their keys in [kFPend, 2 kFPend)) and the direct list of
+    // attended tokens in [2 kFPend, kFBins)
     uint32_t hist[kFBins];
     // one entry per token of the chunk, in token order (entry p: token t0 + p,
-    // scored by thread p mod 256): its bin + 1 (0: no token), bit 15 set once
-    // the token is selected.  Holds the codebook before scoring.
+    // scored by thread p mod 256): its bin + 1 (0: no token) in bits 0-13,
+    // bit 15 set once the token is above the segment's threshold bin, bit 14
+    // once it wins in the threshold bin.  Holds the codebook before scoring.
     alignas(16) uint16_t bins[kFMaxChunk];
     uint32_t rowcnt[kFMaxChunk / 256];        // selected tokens per row of 256, then their prefix
     uint32_t wtot[kFW + 1];
+    uint32_t wcnt[kFW];                       // tokens in each warp's direct list
     uint32_t sc[16];
     float bin_lo, bin_inv;
     int bin_flat, last;
@@ -121,6 +130,7 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 }
 
 // Thread 0 waits until *ctr >= target (bounded); the CTA then synchronizes.
+// The acquire load orders every later read of the CTA after the arrivals.
 __device__ __forceinline__ void cta_wait(const int *ctr, int target, int32_t *status) {
     if (threadIdx.x == 0) {
         int it = 0;
@@ -129,20 +139,22 @@ __device__ __forceinline__ void cta_wait(const int *ctr, int target, int32_t *st
                 flag_error(status, SIKV_DEVERR_TIMEOUT);
                 break;
             }
-            __nanosleep(128);
+            __nanosleep(64);
         }
     }
     __syncthreads();
-    __threadfence();
 }
 
-// Every thread's prior global writes become visible, then thread 0 arrives.
-// Returns the counter's previous value to thread 0 (others get 0).
+// After the CTA barrier thread 0 fences (cumulative over the writes of the
+// CTA that the barrier ordered before it) and arrives.  Returns the
+// counter's previous value to thread 0 (others get 0).
 __device__ __forceinline__ int cta_arrive(int *ctr) {
-    __threadfence();
     __syncthreads();
     int old = 0;
-    if (threadIdx.x == 0) old = atomicAdd(ctr, 1);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        old = atomicAdd(ctr, 1);
+    }
     return old;
 }
 
@@ -230,26 +242,187 @@ __device__ __noinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, u
     return prefix;
 }
 
-// Appends token t of the threshold bin to the segment's candidate list with
-// its exact key: re-scored by the lane that scored it (same table, same
-// rotation, same order of additions, so bit-identical).
-__device__ __noinline__ void emit_candidate(const float *t2, const uint4 *crow, int t, int lane, float qmu,
-                                            int *ncand, uint2 *cand, int cap) {
-    const float sv = lut2_score(t2, __ldg(crow + t), lane, qmu);
-    const int slot = atomicAdd(ncand, 1);
-    if (slot < cap) cand[slot] = make_uint2(score_key(sv), static_cast<uint32_t>(t));
-}
-
 // bins[] holds one 16-bit entry per token of the chunk in token order (entry
 // p is token t0 + p).  A lane scans 8 consecutive entries with one 16-byte
 // load; these give, per 16-bit half of each word, an all-ones mask where the
 // entry's bin is above / equal to a threshold (entries hold bin + 1).
-__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return __vcmpgtu2(w & 0x7FFF7FFFu, thr2); }
-__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) { return __vcmpeq2(w & 0x7FFF7FFFu, thr2); }
+__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return __vcmpgtu2(w & 0x3FFF3FFFu, thr2); }
+__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) { return __vcmpeq2(w & 0x3FFF3FFFu, thr2); }
 // 8-bit mask (bit j = entry j of the lane's 8) from four per-half masks
 __device__ __forceinline__ uint32_t mask8(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
     return (m0 & 1u) | ((m0 >> 15) & 2u) | ((m1 & 1u) << 2) | ((m1 >> 13) & 8u) | ((m2 & 1u) << 4) |
            ((m2 >> 11) & 32u) | ((m3 & 1u) << 6) | ((m3 >> 9) & 128u);
+}
+
+// Appends the tokens of bin b* (entries equal to b2 in both halves) to the
+// segment's candidate list one by one with their exact keys, each re-scored
+// by the lane that scored it (same table, same rotation, same order of
+// additions, so bit-identical).  The fallback for a CTA whose threshold bin
+// holds more tokens than the shared list takes; ties-heavy tables only.
+__device__ __noinline__ void emit_bin_tokens(const uint16_t *bins, int nrows, uint32_t b2, const float *t2,
+                                             const uint4 *crow, int t0, float qmu, int *ncand, uint2 *cand, int cap) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll 1
+    for (int row = warp; row < nrows; row += kFW) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
+        const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
+        // token t0 + p was scored by lane p mod 32 (the table's bank rotation)
+        uint32_t todo = __ballot_sync(0xffffffffu, eq != 0);
+        while (todo) {
+            const int src = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const uint32_t em = __shfl_sync(0xffffffffu, eq, src);
+            for (uint32_t mm = em; mm; mm &= mm - 1) {
+                const int p = row * kFRow + 8 * src + __ffs(mm) - 1;
+                if (lane == (p & 31)) {
+                    const float sv = lut2_score(t2, __ldg(crow + t0 + p), lane, qmu);
+                    const int slot = atomicAdd(ncand, 1);
+                    if (slot < cap) cand[slot] = make_uint2(score_key(sv), static_cast<uint32_t>(t0 + p));
+                }
+            }
+        }
+    }
+}
+
+// Turns sh.rowcnt-style per-row counts into exclusive prefix sums in place and
+// returns the total.  Expects the counts to be visible; ends synchronized.
+__device__ __forceinline__ uint32_t rows_to_bases(uint32_t *rowcnt, int nrows, uint32_t *wtot) {
+    uint32_t total;
+    const int tid = threadIdx.x;
+    const uint32_t v = tid < nrows ? rowcnt[tid] : 0u;
+    const uint32_t run = cta_excl_scan(v, wtot, &total);
+    if (tid < nrows) rowcnt[tid] = run;
+    __syncthreads();
+    return total;
+}
+
+// 8-bit mask of the entries of row `row` (8 per lane) that carry flag bit2.
+__device__ __forceinline__ uint32_t flagged8(const uint16_t *bins, int row, int lane, uint32_t bit2) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
+    return mask8(__vcmpne2(w.x & bit2, 0u), __vcmpne2(w.y & bit2, 0u), __vcmpne2(w.z & bit2, 0u),
+                 __vcmpne2(w.w & bit2, 0u));
+}
+
+// Fills list[0, wn) with the tokens of the entries flagged bit2 whose
+// ordinals (ascending token order) lie in [wbase, wbase + wn).  The fallback
+// when a pass holds more tokens than the direct list takes.  Ends synchronized.
+// (Inlined: as a call it costs the kernel spills around the call site.)
+__device__ __forceinline__ void stage_flagged(const uint16_t *bins, int nrows, uint32_t bit2, uint32_t wbase, int t0,
+                                           uint32_t *rowcnt, uint32_t *wtot, int32_t *list) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll 1
+    for (int row = warp; row < nrows; row += kFW) {
+        uint32_t cnt = __popc(flagged8(bins, row, lane, bit2));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+        if (lane == 0) rowcnt[row] = cnt;
+    }
+    __syncthreads();
+    rows_to_bases(rowcnt, nrows, wtot);
+#pragma unroll 1
+    for (int row = warp; row < nrows; row += kFW) {
+        const uint32_t m = flagged8(bins, row, lane, bit2);
+        uint32_t incl = __popc(m);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o2;
+        }
+        uint32_t ord = rowcnt[row] + incl - __popc(m);
+        for (uint32_t mm = m; mm; mm &= mm - 1, ++ord) {
+            const int t = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
+            if (ord >= wbase && ord < wbase + kFListCap) list[ord - wbase] = t;
+        }
+    }
+    __syncthreads();
+}
+
+// Online-softmax state of one warp: running max m and sum l per head (equal
+// in every lane) and the lane's four output columns (4 lane .. 4 lane + 3).
+template <int GM>
+struct WarpSoftmax {
+    float m[GM], l[GM], o[GM][4];
+};
+
+// A batch of up to 32 entries, one per lane (logit -INFINITY: no entry).
+// Folds the batch's maximum into m, rescales l and o, adds the batch's
+// weights to l and turns lg into the lane's weight exp(lg - m).
+template <int GM>
+__device__ __forceinline__ void warp_softmax_batch(WarpSoftmax<GM> &s, float (&lg)[GM]) {
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+        float mx = lg[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float mn = fmaxf(s.m[g], mx);
+        const float alpha = (s.m[g] == -INFINITY) ? 0.f : __expf(s.m[g] - mn);
+        const float pr = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - mn);
+        float sum = pr;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        s.l[g] = fmaf(s.l[g], alpha, sum);
+        s.m[g] = mn;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s.o[g][i] *= alpha;
+        lg[g] = pr;
+    }
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+// Waits for this thread's outstanding cp.async copies.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Value rows staged per round by a warp.
+template <int DT>
+struct VStage {
+    static constexpr int kRowBytes = kHeadDim * ElemBytes<DT>::value;
+    static constexpr int kRows = kFVBytes / kRowBytes;      // 16 (bf16) or 8 (fp32)
+};
+
+// Starts copying the value rows of tokens tok[j0 .. j0 + n) into vb (row j
+// at j * kRowBytes), 16 bytes per copy, all in flight at once.
+template <int DT>
+__device__ __forceinline__ void warp_stage_v(char *vb, const int32_t *tok, int j0, int n, const char *vseg,
+                                             int lane) {
+    constexpr int kRowBytes = VStage<DT>::kRowBytes, kChunks = kRowBytes / 16;
+#pragma unroll 1
+    for (int i = lane; i < n * kChunks; i += 32) {
+        const int j = i / kChunks, cc = i % kChunks;
+        cp_async16(vb + j * kRowBytes + 16 * cc,
+                   vseg + static_cast<size_t>(tok[j0 + j]) * kRowBytes + 16 * cc);
+    }
+}
+
+// o += sum over the staged rows j < n of pr_{j0+j} V[row j]; lane l takes
+// columns 4l..4l+3.
+template <int DT, int GM>
+__device__ __forceinline__ void warp_fma_v(WarpSoftmax<GM> &s, const char *vb, const float (&pr)[GM], int j0, int n,
+                                           int lane) {
+    constexpr int kRowBytes = VStage<DT>::kRowBytes;
+#pragma unroll 2
+    for (int j = 0; j < n; ++j) {
+        float4 vv;
+        if (DT == SIKV_DTYPE_BF16) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(vb + j * kRowBytes + 8 * lane);
+            vv = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+        } else {
+            vv = *reinterpret_cast<const float4 *>(vb + j * kRowBytes + 16 * lane);
+        }
+#pragma unroll
+        for (int g = 0; g < GM; ++g) {
+            const float w = __shfl_sync(0xffffffffu, pr[g], j0 + j);
+            s.o[g][0] = fmaf(w, vv.x, s.o[g][0]);
+            s.o[g][1] = fmaf(w, vv.y, s.o[g][1]);
+            s.o[g][2] = fmaf(w, vv.z, s.o[g][2]);
+            s.o[g][3] = fmaf(w, vv.w, s.o[g][3]);
+        }
+    }
 }
 
 // Winners among many candidates (more than the rank path takes): radix
@@ -415,6 +588,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         if (tid == 0) {
             sh.sc[0] = 0;
             sh.sc[1] = 0;
+            sh.sc[8] = 0;     // threshold-bin tokens listed
         }
         __syncthreads();
         cta_find_bin<kFBins / kFT>([&](int i) { return sh.hist[i]; }, static_cast<uint32_t>(k), sh.wtot, sh.sc);
@@ -426,328 +600,354 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         }
     }
     cta_arrive(&ctl->arrive1);
+    // this thread's codebook rows for the per-head LUTs, fetched during the wait
+    constexpr int kCbPer = kSubspaces * kClusters / kFT;
+    float4 cbr[kCbPer];
+    {
+        const float4 *cb = reinterpret_cast<const float4 *>(a.codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
+#pragma unroll
+        for (int i = 0; i < kCbPer; ++i) cbr[i] = __ldg(cb + tid + i * kFT);
+    }
     cta_wait(&ctl->arrive1, a.cps, a.status);
 
-    // ---- 2. segment k-th bin b*; count higher bins, list the tokens of b*
+    // ---- 2. segment k-th bin b*.  Tokens above it are selected outright:
+    // flagged (entry bit 15), listed for the attention and their code and
+    // value rows sent to L2.  Tokens in b* are listed, re-scored together and
+    // appended with their exact keys to the segment's candidates.
+    const int nrows = (a.chunk + kFRow - 1) / kFRow;           // <= 64
+    const uint32_t kSure = 0x80008000u, kWin = 0x40004000u;
     int bstar = kFBins;              // nothing selected when k == 0
-    uint32_t above_bstar = 0;
+    uint32_t above_bstar = 0, n_sure = 0;
+    const char *vseg = static_cast<const char *>(a.V) + kv_seg * kHeadDim * EB;
+    uint32_t *pend = sh.hist;                                        // free: the local histogram is published
+    // each warp's direct list of attended tokens (kFWarpList entries)
+    int32_t *wlist = reinterpret_cast<int32_t *>(sh.hist) + 2 * kFPend + kFWarpList * warp;
+    if (lane == 0) sh.wcnt[warp] = 0;
     if (k > 0) {
         const uint32_t *gh = a.ghist + static_cast<size_t>(seg) * kFBins;
         cta_find_bin<kFBins / kFT>([&](int i) { return __ldcg(gh + i); }, static_cast<uint32_t>(k), sh.wtot, sh.sc);
         bstar = static_cast<int>(sh.sc[0]);
         above_bstar = sh.sc[1];
-        uint32_t mine = 0;
-        uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
         const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
-#pragma unroll 1
-        for (int row = warp; row * kFRow < a.chunk; row += kFW) {
-            const int p0 = row * kFRow + 8 * lane;
-            const uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
-            const uint32_t gt = mask8(half_gt(w.x, b2), half_gt(w.y, b2), half_gt(w.z, b2), half_gt(w.w, b2));
-            const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
-            mine += __popc(gt);
-            // selected for sure: the code and value rows are needed by the
-            // attention pass, so they go to L2 now
-            for (uint32_t mm = gt; mm; mm &= mm - 1) {
-                const int t = t0 + p0 + __ffs(mm) - 1;
-                prefetch_l2(crow + t);
-                prefetch_l2(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB);
-                if (EB * kHeadDim > 128) prefetch_l2(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB + 128);
-            }
-            // tokens of the threshold bin: exact key needed.  The lane that
-            // scored token t0 + p is p mod 32 (the table's bank rotation), so
-            // the warp hands each one to that lane.
-            uint32_t todo = __ballot_sync(0xffffffffu, eq != 0);
-            while (todo) {
-                const int src = __ffs(todo) - 1;
-                todo &= todo - 1;
-                const uint32_t em = __shfl_sync(0xffffffffu, eq, src);
-                for (uint32_t mm = em; mm; mm &= mm - 1) {
-                    const int p = row * kFRow + 8 * src + __ffs(mm) - 1;
-                    if (lane == (p & 31))
-                        emit_candidate(sh.u.tab.t2, crow, t0 + p, lane, qmu, &ctl->ncand, cand, a.cand_cap);
-                }
-            }
-        }
-        uint32_t tot;
-        cta_excl_scan(mine, sh.wtot, &tot);
-        if (tid == 0) a.selcnt[static_cast<size_t>(seg) * a.cps + c] = static_cast<int32_t>(tot);
-    }
-    cta_arrive(&ctl->arrive2);
-
-    // Tokens above b* are selected whatever the candidates decide, so they
-    // (and this CTA's share of the sinks) are attended first, while the
-    // other CTAs finish the candidate list; the winners of the threshold bin
-    // follow in a second pass over the same code, continuing the same online
-    // softmax.  Entry bit 15 marks a token of the first pass, bit 14 one of
-    // the second.
-    const int nrows = (a.chunk + kFRow - 1) / kFRow;           // <= 64
-    const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
-    auto row_mask = [&](int row, uint32_t bit2) -> uint32_t {
-        const uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + row * kFRow + 8 * lane);
-        return mask8(__vcmpne2(w.x & bit2, 0u), __vcmpne2(w.y & bit2, 0u), __vcmpne2(w.z & bit2, 0u),
-                     __vcmpne2(w.w & bit2, 0u));
-    };
-    // sets bit2 on the entries picked by pick(row, words) and counts them per row;
-    // returns the total, with sh.rowcnt turned into each row's ordinal base
-    auto mark_rows = [&](uint32_t bit2, auto pick) -> uint32_t {
+        uint32_t n_w = 0;
 #pragma unroll 1
         for (int row = warp; row < nrows; row += kFW) {
             const int p0 = row * kFRow + 8 * lane;
             uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
-            const uint32_t m = pick(p0, w);
-            if (m) {
-                const uint32_t lo = bit2 & 0xFFFFu, hi = bit2 & 0xFFFF0000u;
-                w.x |= ((m & 1u) ? lo : 0u) | ((m & 2u) ? hi : 0u);
-                w.y |= ((m & 4u) ? lo : 0u) | ((m & 8u) ? hi : 0u);
-                w.z |= ((m & 16u) ? lo : 0u) | ((m & 32u) ? hi : 0u);
-                w.w |= ((m & 64u) ? lo : 0u) | ((m & 128u) ? hi : 0u);
+            const uint32_t gx = half_gt(w.x, b2), gy = half_gt(w.y, b2), gz = half_gt(w.z, b2), gw = half_gt(w.w, b2);
+            const uint32_t gt = mask8(gx, gy, gz, gw);
+            const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
+            if (gt) {
+                w.x |= gx & kSure;
+                w.y |= gy & kSure;
+                w.z |= gz & kSure;
+                w.w |= gw & kSure;
                 *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
             }
-            uint32_t cnt = __popc(m);
+            // this warp's list, in row order then token order
+            const uint32_t ng = __popc(gt);
+            uint32_t incl = ng;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-            if (lane == 0) sh.rowcnt[row] = cnt;
-        }
-        __syncthreads();
-        uint32_t total;
-        const uint32_t v = tid < nrows ? sh.rowcnt[tid] : 0u;
-        const uint32_t run = cta_excl_scan(v, sh.wtot, &total);
-        if (tid < nrows) sh.rowcnt[tid] = run;
-        __syncthreads();
-        return total;
-    };
-    const uint32_t kSure = 0x80008000u, kWin = 0x40004000u;
-    const uint32_t n_sure = k > 0 ? mark_rows(kSure, [&](int, uint4 w) -> uint32_t {
-        return mask8(half_gt(w.x, b2), half_gt(w.y, b2), half_gt(w.z, b2), half_gt(w.w, b2));
-    }) : 0u;
-
-    // per-head LUTs: q_h[4s:4s+4] . c[s][j] (the codebook again, from L2)
-    {
-        const float4 *cb = reinterpret_cast<const float4 *>(a.codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
-#pragma unroll 1
-        for (int r = tid; r < kSubspaces * kClusters; r += kFT) {
-            const int s = r >> 4;
-            const float4 c4 = __ldg(cb + r);
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                float v = sh.qs[g][4 * s] * c4.x;
-                v = fmaf(sh.qs[g][4 * s + 1], c4.y, v);
-                v = fmaf(sh.qs[g][4 * s + 2], c4.z, v);
-                v = fmaf(sh.qs[g][4 * s + 3], c4.w, v);
-                sh.u.at.luth[r][g] = v;
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o2;
+            }
+            uint32_t pos = n_w + incl - ng;
+            n_w += __shfl_sync(0xffffffffu, incl, 31);
+            for (uint32_t mm = gt; mm; mm &= mm - 1, ++pos) {
+                const int t = t0 + p0 + __ffs(mm) - 1;
+                if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
+                prefetch_l2(crow + t);
+                prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
+                if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+            }
+            for (uint32_t mm = eq; mm; mm &= mm - 1) {
+                const uint32_t slot = atomicAdd(&sh.sc[8], 1u);
+                if (slot < kFPend) pend[slot] = static_cast<uint32_t>(p0 + __ffs(mm) - 1);
             }
         }
-    }
-    const int n_sinks = min(a.num_sinks, n_tok);
-    const int my_sinks = (n_sinks > c) ? (n_sinks - c + a.cps - 1) / a.cps : 0;   // sinks t = c (mod cps)
-    if (tid < GM) {
-        sh.run_m[tid] = -INFINITY;
-        sh.run_l[tid] = 0.f;
-    }
-    float o[GM][4];
+        if (lane == 0) sh.wcnt[warp] = n_w;
+        __syncthreads();
+        n_sure = 0;
 #pragma unroll
-    for (int g = 0; g < GM; ++g) o[g][0] = o[g][1] = o[g][2] = o[g][3] = 0.f;
-    uint32_t win_before = 0;           // this thread's share of winners with token < t0
-    uint32_t n_win = 0;
+        for (int w2 = 0; w2 < kFW; ++w2) n_sure += sh.wcnt[w2];
+        if (tid == 0) a.selcnt[static_cast<size_t>(seg) * a.cps + c] = static_cast<int32_t>(n_sure);
+        const uint32_t npend = sh.sc[8];
+        uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
+        if (npend <= static_cast<uint32_t>(kFPend)) {
+            // one slot reservation for the CTA, issued before the re-scoring
+            int cbase = 0;
+            if (tid == 0 && npend > 0) cbase = atomicAdd(&ctl->ncand, static_cast<int>(npend));
+            // token t0 + p was scored by lane p mod 32 (the table's bank
+            // rotation): warp e mod 8 takes pending token e in that lane
+#pragma unroll 1
+            for (uint32_t e = warp; e < npend; e += kFW) {
+                const int p = static_cast<int>(pend[e]);
+                if (lane == (p & 31))
+                    pend[kFPend + e] = score_key(lut2_score(sh.u.tab.t2, __ldg(crow + t0 + p), lane, qmu));
+            }
+            if (tid == 0) sh.sc[9] = static_cast<uint32_t>(cbase);
+            __syncthreads();
+            const uint32_t base0 = sh.sc[9];
+            for (uint32_t e = tid; e < npend; e += kFT)
+                if (base0 + e < static_cast<uint32_t>(a.cand_cap))
+                    cand[base0 + e] = make_uint2(pend[kFPend + e], static_cast<uint32_t>(t0) + pend[e]);
+        } else {
+            emit_bin_tokens(sh.bins, nrows, b2, sh.u.tab.t2, crow, t0, qmu, &ctl->ncand, cand, a.cand_cap);
+        }
+    }
+    cta_arrive(&ctl->arrive2);
 
+    // Attention.  Each warp keeps its own online softmax; the warps' states
+    // merge once at the end.  The sinks and the tokens above b* need no
+    // candidate ranking, so they are attended while the other CTAs finish
+    // their candidates; the winners of b* follow after the wait.
+    // The sinks t = c (mod cps): one warp per sink, lane l takes columns
+    // 4l..4l+3 of its stored key and value.  The first sink's rows are
+    // fetched before the LUTs are built.
+    const int n_sinks = min(a.num_sinks, n_tok);
+    const int my_sinks = (n_sinks > c) ? (n_sinks - c + a.cps - 1) / a.cps : 0;
+    const char *kseg = static_cast<const char *>(a.K) + kv_seg * kHeadDim * EB;
+    float4 sk_k = make_float4(0.f, 0.f, 0.f, 0.f), sk_v = sk_k;
+    if (warp < my_sinks) {
+        const size_t off = static_cast<size_t>(c + warp * a.cps) * kHeadDim * EB;
+        sk_k = load4<DT>(kseg + off, 4 * lane);
+        sk_v = load4<DT>(vseg + off, 4 * lane);
+    }
+    // per-head LUTs: q_h[4s:4s+4] . c[s][j]
+#pragma unroll
+    for (int i = 0; i < kCbPer; ++i) {
+        const int r = tid + i * kFT, sidx = r >> 4;
+        const float4 c4 = cbr[i];
+#pragma unroll
+        for (int g = 0; g < GM; ++g) {
+            float v = sh.qs[g][4 * sidx] * c4.x;
+            v = fmaf(sh.qs[g][4 * sidx + 1], c4.y, v);
+            v = fmaf(sh.qs[g][4 * sidx + 2], c4.z, v);
+            v = fmaf(sh.qs[g][4 * sidx + 3], c4.w, v);
+            sh.u.at.luth[r][g] = v;
+        }
+    }
+    WarpSoftmax<GM> ws;
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+        ws.m[g] = -INFINITY;
+        ws.l[g] = 0.f;
+        ws.o[g][0] = ws.o[g][1] = ws.o[g][2] = ws.o[g][3] = 0.f;
+    }
+#pragma unroll 1
+    for (int i = warp; i < my_sinks; i += kFW) {
+        if (i != warp) {
+            const size_t off = static_cast<size_t>(c + i * a.cps) * kHeadDim * EB;
+            sk_k = load4<DT>(kseg + off, 4 * lane);
+            sk_v = load4<DT>(vseg + off, 4 * lane);
+        }
+#pragma unroll
+        for (int g = 0; g < GM; ++g) {
+            float d = sh.qs[g][4 * lane] * sk_k.x;
+            d = fmaf(sh.qs[g][4 * lane + 1], sk_k.y, d);
+            d = fmaf(sh.qs[g][4 * lane + 2], sk_k.z, d);
+            d = fmaf(sh.qs[g][4 * lane + 3], sk_k.w, d);
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
+            const float lgv = (g < group) ? d * a.scale : -INFINITY;
+            const float mn = fmaxf(ws.m[g], lgv);
+            const float alpha = (ws.m[g] == -INFINITY) ? 0.f : __expf(ws.m[g] - mn);
+            const float pr = (lgv == -INFINITY) ? 0.f : __expf(lgv - mn);
+            ws.l[g] = fmaf(ws.l[g], alpha, pr);
+            ws.m[g] = mn;
+            ws.o[g][0] = fmaf(pr, sk_v.x, ws.o[g][0] * alpha);
+            ws.o[g][1] = fmaf(pr, sk_v.y, ws.o[g][1] * alpha);
+            ws.o[g][2] = fmaf(pr, sk_v.z, ws.o[g][2] * alpha);
+            ws.o[g][3] = fmaf(pr, sk_v.w, ws.o[g][3] * alpha);
+        }
+    }
+    __syncthreads();
+    uint32_t win_before = 0;           // this thread's share of winners with token < t0
+    // Each warp attends its own direct list (deterministic order) unless some
+    // warp's list overflowed; then the pass's tokens are staged from the
+    // entry flags in windows of kFListCap and shared out 8 lanes apart.
+    bool direct = true;
+    for (int w2 = 0; w2 < kFW; ++w2) direct = direct && sh.wcnt[w2] <= static_cast<uint32_t>(kFWarpList);
+    uint32_t n_list = n_sure, bit2 = kSure;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
-        uint32_t n_sel = n_sure, bit2 = kSure, n_list = n_sure + static_cast<uint32_t>(my_sinks);
-        if (pass == 1) {
+        int pass_v = pass;
+        asm volatile("" : "+r"(pass_v));   // keeps the two passes in one copy of the code
+        if (pass_v == 1) {
+            if (k == 0) break;
             // ---- exact winners among the threshold-bin candidates (the same
             // answer in every CTA): a candidate wins when fewer than `need`
-            // candidates come before it (key descending, token ascending)
+            // candidates come before it (key descending, token ascending).
+            // The count and the first 2 kFT entries are read together; entries
+            // past the count are ignored.
             cta_wait(&ctl->arrive2, a.cps, a.status);
+            const uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
+            const int nc_raw = __ldcg(&ctl->ncand);
+            const uint2 zero2 = make_uint2(0u, 0u);
+            const uint2 c0 = (tid < a.cand_cap) ? __ldcg(cand + tid) : zero2;
+            const uint2 c1 = (tid + kFT < a.cand_cap) ? __ldcg(cand + tid + kFT) : zero2;
+            const int ncand = min(nc_raw, a.cand_cap);
+            const uint32_t need = static_cast<uint32_t>(k) - above_bstar;   // >= 1
+            const bool ranked = ncand <= kFRankMax;
             for (int i = tid; i < kFMaxChunk / 32; i += kFT) sh.u.sel.winbits[i] = 0;
-            __syncthreads();
-            if (k > 0) {
-                const int ncand = min(__ldcg(&ctl->ncand), a.cand_cap);
-                const uint2 *cand = a.cand + static_cast<size_t>(seg) * a.cand_cap;
-                const uint32_t need = static_cast<uint32_t>(k) - above_bstar;   // >= 1
-                if (ncand <= kFRankMax) {
-                    for (int e = tid; e < ncand; e += kFT) {
-                        const uint2 v = __ldcg(cand + e);
-                        sh.u.sel.ckey[e] = v.x;
-                        sh.u.sel.cidx[e] = static_cast<int32_t>(v.y);
-                    }
-                    __syncthreads();
-                    for (int e = tid; e < ncand; e += kFT) {
-                        const uint32_t ke = sh.u.sel.ckey[e], ie = static_cast<uint32_t>(sh.u.sel.cidx[e]);
-                        uint32_t rank = 0;
-                        for (int f = 0; f < ncand; ++f) {
-                            const uint32_t kf = sh.u.sel.ckey[f];
-                            rank += (kf > ke) || (kf == ke && static_cast<uint32_t>(sh.u.sel.cidx[f]) < ie);
-                        }
-                        if (rank < need) {
-                            const int rel = static_cast<int>(ie) - t0;
-                            if (rel >= 0 && rel < a.chunk) atomicOr(&sh.u.sel.winbits[rel >> 5], 1u << (rel & 31));
-                            else if (rel < 0) ++win_before;
-                        }
-                    }
-                } else {
-                    win_before += refine_by_radix(cand, ncand, need, t0, a.chunk, sh.u.sel.winbits, sh.hist, sh.wtot,
-                                                  sh.sc);
+            if (ranked) {
+                if (tid < ncand) {
+                    sh.u.sel.ckey[tid] = c0.x;
+                    sh.u.sel.cidx[tid] = static_cast<int32_t>(c0.y);
                 }
-                __syncthreads();
-                n_win = mark_rows(kWin, [&](int p0, uint4 w) -> uint32_t {
-                    const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
-                    return eq ? (eq & ((sh.u.sel.winbits[p0 >> 5] >> (p0 & 31)) & 0xFFu)) : 0u;
-                });
+                if (tid + kFT < ncand) {
+                    sh.u.sel.ckey[tid + kFT] = c1.x;
+                    sh.u.sel.cidx[tid + kFT] = static_cast<int32_t>(c1.y);
+                }
             }
-            n_sel = n_win;
+            __syncthreads();
+            if (ranked) {
+                for (int e = tid; e < ncand; e += kFT) {
+                    const uint32_t ke = sh.u.sel.ckey[e], ie = static_cast<uint32_t>(sh.u.sel.cidx[e]);
+                    uint32_t rank = 0;
+#pragma unroll 4
+                    for (int f = 0; f < ncand; ++f) {
+                        const uint32_t kf = sh.u.sel.ckey[f];
+                        rank += (kf > ke) || (kf == ke && static_cast<uint32_t>(sh.u.sel.cidx[f]) < ie);
+                    }
+                    if (rank < need) {
+                        const int rel = static_cast<int>(ie) - t0;
+                        if (rel >= 0 && rel < a.chunk) atomicOr(&sh.u.sel.winbits[rel >> 5], 1u << (rel & 31));
+                        else if (rel < 0) ++win_before;
+                    }
+                }
+            } else {
+                win_before += refine_by_radix(cand, ncand, need, t0, a.chunk, sh.u.sel.winbits, sh.hist, sh.wtot,
+                                              sh.sc);
+            }
+            __syncthreads();
+            // each warp lists the winners of its share of the chunk's bitmap,
+            // in ascending token order
+            {
+                const int nwords = (a.chunk + 31) / 32;
+                const int wpw = (nwords + kFW - 1) / kFW;        // <= 64
+                uint32_t n_w = 0;
+#pragma unroll 1
+                for (int i0 = 0; i0 < wpw; i0 += 32) {
+                    const int wd = warp * wpw + i0 + lane;
+                    const uint32_t bits = (i0 + lane < wpw && wd < nwords) ? sh.u.sel.winbits[wd] : 0u;
+                    const uint32_t cb = __popc(bits);
+                    uint32_t incl = cb;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (lane >= off) incl += o2;
+                    }
+                    uint32_t pos = n_w + incl - cb;
+                    n_w += __shfl_sync(0xffffffffu, incl, 31);
+                    for (uint32_t mm = bits; mm; mm &= mm - 1, ++pos)
+                        if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t0 + 32 * wd + __ffs(mm) - 1;
+                }
+                if (lane == 0) sh.wcnt[warp] = n_w;
+            }
+            __syncthreads();
+            direct = true;
+            n_list = 0;
+            for (int w2 = 0; w2 < kFW; ++w2) {
+                direct = direct && sh.wcnt[w2] <= static_cast<uint32_t>(kFWarpList);
+                n_list += sh.wcnt[w2];
+            }
             bit2 = kWin;
-            n_list = n_win;
+            if (!direct || a.idx_out) {
+                // flag the winners of this chunk (entry bit 14)
+                const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
+#pragma unroll 1
+                for (int row = warp; row < nrows; row += kFW) {
+                    const int p0 = row * kFRow + 8 * lane;
+                    uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
+                    const uint32_t wb = (sh.u.sel.winbits[p0 >> 5] >> (p0 & 31)) & 0xFFu;
+                    // per 16-bit half: all ones where the entry is in b* and won
+                    const uint32_t hx = half_eq(w.x, b2) & (((wb & 1u) ? 0xFFFFu : 0u) | ((wb & 2u) ? 0xFFFF0000u : 0u));
+                    const uint32_t hy = half_eq(w.y, b2) & (((wb & 4u) ? 0xFFFFu : 0u) | ((wb & 8u) ? 0xFFFF0000u : 0u));
+                    const uint32_t hz = half_eq(w.z, b2) & (((wb & 16u) ? 0xFFFFu : 0u) | ((wb & 32u) ? 0xFFFF0000u : 0u));
+                    const uint32_t hw = half_eq(w.w, b2) & (((wb & 64u) ? 0xFFFFu : 0u) | ((wb & 128u) ? 0xFFFF0000u : 0u));
+                    if (hx | hy | hz | hw) {
+                        w.x |= hx & kWin;
+                        w.y |= hy & kWin;
+                        w.z |= hz & kWin;
+                        w.w |= hw & kWin;
+                        *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
+                    }
+                }
+                __syncthreads();
+            }
         }
+        const uint32_t n_windows = direct ? 1u : (n_list + kFListCap - 1) / kFListCap;
 #pragma unroll 1
-        for (uint32_t wbase = 0; wbase < n_list; wbase += kFListCap) {
-            // stage the window [wbase, wbase + kFListCap) of this pass's list:
-            // selected tokens in ascending order, then (first pass) the sinks
-            const uint32_t wn = min(static_cast<uint32_t>(kFListCap), n_list - wbase);
-#pragma unroll 1
-            for (int row = warp; row < nrows; row += kFW) {
-                const uint32_t m = row_mask(row, bit2);
-                uint32_t incl = __popc(m);
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += o2;
-                }
-                uint32_t ord = sh.rowcnt[row] + incl - __popc(m);
-                for (uint32_t mm = m; mm; mm &= mm - 1, ++ord) {
-                    const int t = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
-                    if (ord >= wbase && ord < wbase + kFListCap) sh.u.at.list[ord - wbase] = t;
-                }
+        for (uint32_t win = 0; win < n_windows; ++win) {
+            const int32_t *lst = wlist;
+            uint32_t nl = sh.wcnt[warp], lmul = 1, ladd = 0;
+            if (!direct) {
+                const uint32_t wbase = win * kFListCap;
+                stage_flagged(sh.bins, nrows, bit2, wbase, t0, sh.rowcnt, sh.wtot, sh.u.at.list);
+                lst = sh.u.at.list;
+                nl = min(static_cast<uint32_t>(kFListCap), n_list - wbase);
+                lmul = 8;
+                ladd = static_cast<uint32_t>(warp);
             }
-            for (uint32_t e = tid; e < wn; e += kFT) {
-                const uint32_t ord = wbase + e;
-                if (ord >= n_sel) sh.u.at.list[e] = -1 - static_cast<int32_t>(c + (ord - n_sel) * a.cps);   // a sink
-            }
-            __syncthreads();
+            // opaque to the optimizer: one copy of the batch loop serves both list kinds
+            asm volatile("" : "+l"(lst), "+r"(nl), "+r"(lmul), "+r"(ladd));
+            // batches of up to 32 entries: entry r0 + lmul lane + ladd
 #pragma unroll 1
-            for (uint32_t tbase = 0; tbase < wn; tbase += kFTile) {
-                const uint32_t tile_n = min(static_cast<uint32_t>(kFTile), wn - tbase);
-                // logits, one list entry per thread
-                {
-                    float lg[GM];
+            for (uint32_t r0 = 0; r0 < nl; r0 += 32 * lmul) {
+                const uint32_t e = r0 + lmul * lane + ladd;
+                const bool valid = e < nl;
+                const int nb = __popc(__ballot_sync(0xffffffffu, valid));   // the valid lanes are 0..nb-1
+                if (nb == 0) break;
+                const int t = valid ? lst[e] : 0;
+                const uint4 row = valid ? __ldg(crow + t) : make_uint4(0u, 0u, 0u, 0u);
+                int32_t *tok = sh.u.at.tok[warp];
+                char *vb = sh.u.at.vbuf[warp];
+                tok[lane] = t;
+                __syncwarp();
+                // the first value rows are in flight while the logits are formed
+                constexpr int kVR = VStage<DT>::kRows;
+                warp_stage_v<DT>(vb, tok, 0, min(nb, kVR), vseg, lane);
+                float lg[GM];
 #pragma unroll
-                    for (int g = 0; g < GM; ++g) lg[g] = -INFINITY;
-                    if (static_cast<uint32_t>(tid) < tile_n) {
-                        const int32_t ent = sh.u.at.list[tbase + tid];
-                        float acc[GM];
+                for (int g = 0; g < GM; ++g) lg[g] = -INFINITY;
+                if (valid) {
+                    const uint32_t wd[4] = {row.x, row.y, row.z, row.w};
+                    float acc[GM];
 #pragma unroll
-                        for (int g = 0; g < GM; ++g) acc[g] = 0.f;
-                        if (ent >= 0) {
-                            const uint4 row = __ldg(crow + ent);
-                            const uint32_t w[4] = {row.x, row.y, row.z, row.w};
-#pragma unroll 8
-                            for (int s = 0; s < kSubspaces; ++s) {
-                                const int j = (w[s >> 3] >> (4 * (s & 7))) & 15;
-                                const float *lp = sh.u.at.luth[s * kClusters + j];
+                    for (int g = 0; g < GM; ++g) acc[g] = 0.f;
+#pragma unroll 4
+                    for (int sidx = 0; sidx < kSubspaces; ++sidx) {
+                        const int j = (wd[sidx >> 3] >> (4 * (sidx & 7))) & 15;
+                        const float *lp = sh.u.at.luth[sidx * kClusters + j];
 #pragma unroll
-                                for (int g = 0; g < GM; g += 4) {
-                                    const float4 v4 = *reinterpret_cast<const float4 *>(lp + g);
-                                    acc[g] += v4.x;
-                                    acc[g + 1] += v4.y;
-                                    acc[g + 2] += v4.z;
-                                    acc[g + 3] += v4.w;
-                                }
-                            }
-#pragma unroll
-                            for (int g = 0; g < GM; ++g) lg[g] = (acc[g] + sh.qmu_h[g]) * a.scale;
-                        } else {
-                            const char *krow = static_cast<const char *>(a.K) + (kv_seg + (-1 - ent)) * kHeadDim * EB;
-#pragma unroll 2
-                            for (int d = 0; d < kHeadDim; d += 4) {
-                                const float4 kv = load4<DT>(krow, d);
-#pragma unroll
-                                for (int g = 0; g < GM; ++g) {
-                                    acc[g] = fmaf(sh.qs[g][d], kv.x, acc[g]);
-                                    acc[g] = fmaf(sh.qs[g][d + 1], kv.y, acc[g]);
-                                    acc[g] = fmaf(sh.qs[g][d + 2], kv.z, acc[g]);
-                                    acc[g] = fmaf(sh.qs[g][d + 3], kv.w, acc[g]);
-                                }
-                            }
-#pragma unroll
-                            for (int g = 0; g < GM; ++g) lg[g] = acc[g] * a.scale;
+                        for (int g = 0; g < GM; g += 4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(lp + g);
+                            acc[g] += v4.x;
+                            acc[g + 1] += v4.y;
+                            acc[g + 2] += v4.z;
+                            acc[g + 3] += v4.w;
                         }
                     }
 #pragma unroll
-                    for (int g = 0; g < GM; ++g) {
-                        const float v = (g < group) ? lg[g] : -INFINITY;
-                        sh.u.at.logit[g][tid] = v;
-                        float mx = v;
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                        if (lane == 0) sh.tile_stat[warp][g] = mx;
-                    }
+                    for (int g = 0; g < GM; ++g) lg[g] = (g < group) ? (acc[g] + sh.qmu_h[g]) * a.scale : -INFINITY;
                 }
-                __syncthreads();
-                // new running max per head and the rescale factor of what came before
-                float alpha[GM], mnew[GM];
-#pragma unroll
-                for (int g = 0; g < GM; ++g) {
-                    float mx = sh.run_m[g];
-                    for (int w = 0; w < kFW; ++w) mx = fmaxf(mx, sh.tile_stat[w][g]);
-                    mnew[g] = mx;
-                    alpha[g] = (sh.run_m[g] == -INFINITY) ? 0.f : __expf(sh.run_m[g] - mx);
-                }
-                __syncthreads();
-#pragma unroll
-                for (int g = 0; g < GM; ++g) {
-                    const float lv = sh.u.at.logit[g][tid];
-                    const float pr = (lv == -INFINITY) ? 0.f : __expf(lv - mnew[g]);
-                    sh.u.at.logit[g][tid] = pr;
-                    float sm = pr;
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
-                    if (lane == 0) sh.tile_stat[warp][g] = sm;
-                }
-                __syncthreads();
-                if (tid < GM) {
-                    float sm = 0.f;
-                    for (int w = 0; w < kFW; ++w) sm += sh.tile_stat[w][tid];
-                    sh.run_l[tid] = sh.run_l[tid] * alpha[tid] + sm;
-                    sh.run_m[tid] = mnew[tid];
-                }
-                // o = alpha o + sum_e p_e V[t_e]; warp w takes entries w, w + 8, ...
-#pragma unroll
-                for (int g = 0; g < GM; ++g) {
-                    o[g][0] *= alpha[g];
-                    o[g][1] *= alpha[g];
-                    o[g][2] *= alpha[g];
-                    o[g][3] *= alpha[g];
-                }
+                warp_softmax_batch(ws, lg);
 #pragma unroll 1
-                for (uint32_t e0 = warp; e0 < tile_n; e0 += kFVRows * kFW) {
-                    float4 v[kFVRows];
-#pragma unroll
-                    for (int u = 0; u < kFVRows; ++u) {
-                        const uint32_t e = e0 + u * kFW;
-                        if (e < tile_n) {
-                            const int32_t ent = sh.u.at.list[tbase + e];
-                            const int t = ent >= 0 ? ent : -1 - ent;
-                            v[u] = load4<DT>(static_cast<const char *>(a.V) + (kv_seg + t) * kHeadDim * EB, lane * 4);
-                        } else {
-                            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
+                for (int j0 = 0; j0 < nb; j0 += kVR) {
+                    const int n = min(kVR, nb - j0);
+                    if (j0 > 0) {
+                        __syncwarp();          // every lane is done with the previous rows
+                        warp_stage_v<DT>(vb, tok, j0, n, vseg, lane);
                     }
-#pragma unroll
-                    for (int u = 0; u < kFVRows; ++u) {
-                        const uint32_t e = e0 + u * kFW;
-                        const float4 vv = v[u];
-#pragma unroll
-                        for (int g = 0; g < GM; ++g) {
-                            const float pr = e < tile_n ? sh.u.at.logit[g][e] : 0.f;
-                            o[g][0] = fmaf(pr, vv.x, o[g][0]);
-                            o[g][1] = fmaf(pr, vv.y, o[g][1]);
-                            o[g][2] = fmaf(pr, vv.z, o[g][2]);
-                            o[g][3] = fmaf(pr, vv.w, o[g][3]);
-                        }
-                    }
+                    cp_async_wait_all();
+                    __syncwarp();
+                    warp_fma_v<DT, GM>(ws, vb, lg, j0, n, lane);
                 }
-                __syncthreads();
+                __syncwarp();                  // tok and vbuf are reused by the next batch
             }
+            if (!direct) __syncthreads();
         }
     }
 
@@ -761,24 +961,17 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         cta_excl_scan(before, sh.wtot, &out_base);
 #pragma unroll 1
         for (int row = warp; row < nrows; row += kFW) {
-            const uint32_t m = row_mask(row, kSure | kWin);
-            uint32_t cnt = __popc(m);
+            uint32_t cnt = __popc(flagged8(sh.bins, row, lane, kSure | kWin));
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
             if (lane == 0) sh.rowcnt[row] = cnt;
         }
         __syncthreads();
-        {
-            uint32_t total;
-            const uint32_t v = tid < nrows ? sh.rowcnt[tid] : 0u;
-            const uint32_t run = cta_excl_scan(v, sh.wtot, &total);
-            if (tid < nrows) sh.rowcnt[tid] = run;
-            __syncthreads();
-        }
+        rows_to_bases(sh.rowcnt, nrows, sh.wtot);
         int32_t *io = a.idx_out + static_cast<size_t>(seg) * a.kmax;
 #pragma unroll 1
         for (int row = warp; row < nrows; row += kFW) {
-            const uint32_t m = row_mask(row, kSure | kWin);
+            const uint32_t m = flagged8(sh.bins, row, lane, kSure | kWin);
             uint32_t incl = __popc(m);
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -791,51 +984,95 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         }
     }
 
-    // reduce o over the warps and write this CTA's partial
+    // merge the warps' softmax states into this CTA's partial (m, l, o)
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < GM; ++g) {
+            sh.wm[warp][g] = ws.m[g];
+            sh.wl[warp][g] = ws.l[g];
+        }
+    }
 #pragma unroll
     for (int g = 0; g < GM; ++g)
-        *reinterpret_cast<float4 *>(&sh.u.at.red[warp][g][lane * 4]) = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+        *reinterpret_cast<float4 *>(&sh.u.at.red[warp][g][lane * 4]) =
+            make_float4(ws.o[g][0], ws.o[g][1], ws.o[g][2], ws.o[g][3]);
     __syncthreads();
     {
         const size_t pb = (static_cast<size_t>(seg) * a.cps + c) * GM;
         for (int e = tid; e < GM * kHeadDim; e += kFT) {
             const int g = e / kHeadDim, d = e % kHeadDim;
-            float s = sh.u.at.red[0][g][d];
+            float mx = -INFINITY;
 #pragma unroll
-            for (int w = 1; w < kFW; ++w) s += sh.u.at.red[w][g][d];
-            a.part_o[(pb + g) * kHeadDim + d] = s;
+            for (int w = 0; w < kFW; ++w) mx = fmaxf(mx, sh.wm[w][g]);
+            float sacc = 0.f, lsum = 0.f;
+            if (mx != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kFW; ++w) {
+                    const float mw = sh.wm[w][g];
+                    const float f = (mw == -INFINITY) ? 0.f : __expf(mw - mx);
+                    sacc = fmaf(f, sh.u.at.red[w][g][d], sacc);
+                    lsum = fmaf(f, sh.wl[w][g], lsum);
+                }
+            }
+            a.part_o[(pb + g) * kHeadDim + d] = sacc;
+            if (d == 0) a.part_ml[pb + g] = make_float2(mx, lsum);
         }
-        if (tid < GM) a.part_ml[pb + tid] = make_float2(sh.run_m[tid], sh.run_l[tid]);
     }
 
-    // ---- last CTA of the segment: merge partials, reset coordination state
+    // ---- last CTA of the segment: merge the partials, reset the coordination state
     const int old = cta_arrive(&ctl->arrive3);
     if (tid == 0) sh.last = (old == a.cps - 1);
     __syncthreads();
     if (!sh.last) return;
     __threadfence();
-#pragma unroll 1
-    for (int e = tid; e < group * kHeadDim; e += kFT) {
-        const int g = e / kHeadDim, d = e % kHeadDim;
-        float mx = -INFINITY;
-        for (int cc = 0; cc < a.cps; ++cc)
-            mx = fmaxf(mx, __ldcg(a.part_ml + (static_cast<size_t>(seg) * a.cps + cc) * GM + g).x);
-        float l = 0.f, acc = 0.f;
-        if (mx != -INFINITY) {
-            for (int cc = 0; cc < a.cps; ++cc) {
-                const size_t pb = (static_cast<size_t>(seg) * a.cps + cc) * GM + g;
-                const float2 ml = __ldcg(a.part_ml + pb);
-                const float wgt = (ml.x == -INFINITY) ? 0.f : __expf(ml.x - mx);
-                l = fmaf(ml.y, wgt, l);
-                acc = fmaf(__ldcg(a.part_o + pb * kHeadDim + d), wgt, acc);
-            }
+    {
+        // this thread's output elements e = tid + kFT i; the first kFPre
+        // partials of each are fetched together with the (m, l) pairs
+        constexpr int kEl = GM * kHeadDim / kFT;       // 2 or 4
+        constexpr int kFPre = kEl == 2 ? 16 : 8;
+        const size_t seg_p = static_cast<size_t>(seg) * a.cps;
+        float pre[kEl][kFPre];
+#pragma unroll
+        for (int i = 0; i < kEl; ++i) {
+            const int e = tid + kFT * i, g = e / kHeadDim, d = e % kHeadDim;
+#pragma unroll
+            for (int cc = 0; cc < kFPre; ++cc)
+                pre[i][cc] = (g < group && cc < a.cps) ? __ldcg(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d) : 0.f;
         }
-        const float r = (l > 0.f) ? __fdividef(acc, l) : 0.f;
-        const size_t orow = (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group + g) * kHeadDim + d;
-        if (DT == SIKV_DTYPE_F32)
-            static_cast<float *>(a.out)[orow] = r;
-        else
-            static_cast<unsigned short *>(a.out)[orow] = static_cast<unsigned short>(f32_to_bf16_bits(r));
+        float2 *mls = reinterpret_cast<float2 *>(&sh.u.at.red[0][0][0]);       // [cps][GM]
+        float *wts = reinterpret_cast<float *>(mls + kFusedMaxCps * GM);       // [cps][GM]
+        for (int e = tid; e < a.cps * GM; e += kFT) mls[e] = __ldcg(a.part_ml + seg_p * GM + e);
+        __syncthreads();
+        if (tid < GM) {
+            float mx = -INFINITY;
+            for (int cc = 0; cc < a.cps; ++cc) mx = fmaxf(mx, mls[cc * GM + tid].x);
+            float l = 0.f;
+            for (int cc = 0; cc < a.cps; ++cc) {
+                const float2 ml = mls[cc * GM + tid];
+                const float f = (ml.x == -INFINITY) ? 0.f : __expf(ml.x - mx);
+                wts[cc * GM + tid] = f;
+                l = fmaf(ml.y, f, l);
+            }
+            const float inv = (l > 0.f) ? __fdividef(1.f, l) : 0.f;
+            for (int cc = 0; cc < a.cps; ++cc) wts[cc * GM + tid] *= inv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kEl; ++i) {
+            const int e = tid + kFT * i, g = e / kHeadDim, d = e % kHeadDim;
+            if (g >= group) continue;
+            float acc = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < kFPre; ++cc) acc = fmaf(wts[min(cc, a.cps - 1) * GM + g], pre[i][cc], acc);
+#pragma unroll 4
+            for (int cc = kFPre; cc < a.cps; ++cc)
+                acc = fmaf(wts[cc * GM + g], __ldcg(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d), acc);
+            const size_t orow = (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group + g) * kHeadDim + d;
+            if (DT == SIKV_DTYPE_F32)
+                static_cast<float *>(a.out)[orow] = acc;
+            else
+                static_cast<unsigned short *>(a.out)[orow] = static_cast<unsigned short>(f32_to_bf16_bits(acc));
+        }
     }
     if (a.idx_out) {
         int32_t *io = a.idx_out + static_cast<size_t>(seg) * a.kmax;
