@@ -45,10 +45,9 @@ constexpr int kFBins = 1024;             // histogram bins per segment
 constexpr int kFListCap = 2048;          // attended tokens staged per window
 constexpr int kFMaxNpt = 64;             // token slots per thread at most
 constexpr int kFMaxChunk = kFMaxNpt * kFT;
-constexpr int kFCandSmem = 1024;         // candidates staged in shared memory
 constexpr int kFRankMax = 512;           // up to this many candidates: rank directly
 constexpr int kFUnroll = 8;              // code rows in flight per thread
-constexpr int kFPrefetchRows = 16;       // code rows per thread kept ahead in L2
+constexpr int kFPrefetchRows = 16;       // code rows per thread sent to L2 during the prologue
 constexpr int kFPend = kFBins / 4;       // threshold-bin tokens of a CTA re-scored together
 constexpr int kFDirect = kFBins / 2;     // attended tokens listed directly during the scans
 constexpr int kFWarpList = kFDirect / kFW;   // of which each warp lists (and attends) at most this many
@@ -83,8 +82,9 @@ struct FusedSmem {
     union {
         ScoreTables tab;
         struct {
-            uint32_t ckey[kFCandSmem];
-            int32_t cidx[kFCandSmem];
+            // candidate (key, token) as one 64-bit value: key above the
+            // inverted token, so a larger value ranks first (ties: lower token)
+            unsigned long long ck[kFRankMax];
             uint32_t winbits[kFMaxChunk / 32];
         } sel;
         struct {
@@ -480,8 +480,11 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     const uint4 *crow = reinterpret_cast<const uint4 *>(a.codes) + kv_seg;
     const int my = 32 * warp + lane;                         // slot i of this thread: token t0 + 256 i + my
 
-    // ---- tables.  The prologue leaves HBM idle, so the first code rows and
-    // this CTA's share of the sink rows go to L2 meanwhile.
+    // ---- tables.  Their inputs are requested first; while they travel, the
+    // first code rows and this CTA's share of the sink rows go to L2 (the
+    // prologue would otherwise leave HBM idle).
+    TableInputs<DT> tin;
+    tin.load(a.q, a.codebook, a.mu, b, h, a.hq, group, seg);
 #pragma unroll 1
     for (int i = 0; i < kFPrefetchRows && i < npt; ++i) {
         const int t = t0 + kFT * i + my;
@@ -496,9 +499,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     }
     float4 *cbs = reinterpret_cast<float4 *>(sh.bins);     // 8 KB, free until scoring
     for (int e = tid; e < GM * kHeadDim; e += kFT) sh.qs[e / kHeadDim][e % kHeadDim] = 0.f;
-    __syncthreads();
-    stage_table_inputs<DT>(&sh.qs[0][0], cbs, sh.mus, a.q, a.codebook, a.mu, b, h, a.hq, group, seg);
     for (int i = tid; i < kFBins; i += kFT) sh.hist[i] = 0;
+    __syncthreads();
+    tin.store(&sh.qs[0][0], cbs, sh.mus, group);
     __syncthreads();
     build_score_tables(sh.u.tab, &sh.qs[0][0], cbs, sh.mus, group);
     for (int g = warp; g < GM; g += kFW) {
@@ -541,18 +544,23 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     // ---- scores of this chunk -> histogram and per-slot bins
     {
         float *so = a.scores_out ? a.scores_out + kv_seg : nullptr;
+        // rows of the next group are requested before the current group is
+        // scored, so each thread always has a group of rows in flight
+        uint4 nxt[kFUnroll];
+#pragma unroll
+        for (int u = 0; u < kFUnroll; ++u) {
+            const int t = t0 + kFT * u + my;
+            nxt[u] = (u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll 1
         for (int i0 = 0; i0 < npt; i0 += kFUnroll) {
-#pragma unroll
-            for (int u = 0; u < kFUnroll; ++u) {
-                const int t = t0 + kFT * (i0 + kFPrefetchRows + u) + my;
-                if (i0 + kFPrefetchRows + u < npt && t >= tstart && t < t1) prefetch_l2(crow + t);
-            }
             uint4 rows[kFUnroll];
 #pragma unroll
+            for (int u = 0; u < kFUnroll; ++u) rows[u] = nxt[u];
+#pragma unroll
             for (int u = 0; u < kFUnroll; ++u) {
-                const int t = t0 + kFT * (i0 + u) + my;
-                rows[u] = (i0 + u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
+                const int t = t0 + kFT * (i0 + kFUnroll + u) + my;
+                nxt[u] = (i0 + kFUnroll + u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
             }
             float sc2[kFUnroll];
 #pragma unroll
@@ -629,6 +637,10 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         bstar = static_cast<int>(sh.sc[0]);
         above_bstar = sh.sc[1];
         const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
+        // warp w scans rows w, w + 8, ... of 256 entries (8 per lane) and lists
+        // its tokens in ascending order; list positions come from one ballot
+        // per entry slot, not from a shuffle scan
+        const uint32_t below = (1u << lane) - 1u;
         uint32_t n_w = 0;
 #pragma unroll 1
         for (int row = warp; row < nrows; row += kFW) {
@@ -637,33 +649,32 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
             const uint32_t gx = half_gt(w.x, b2), gy = half_gt(w.y, b2), gz = half_gt(w.z, b2), gw = half_gt(w.w, b2);
             const uint32_t gt = mask8(gx, gy, gz, gw);
             const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
+            uint32_t pos = n_w;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t bj = __ballot_sync(0xffffffffu, (gt >> j) & 1u);
+                pos += __popc(bj & below);
+                n_w += __popc(bj);
+            }
             if (gt) {
                 w.x |= gx & kSure;
                 w.y |= gy & kSure;
                 w.z |= gz & kSure;
                 w.w |= gw & kSure;
                 *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
-            }
-            // this warp's list, in row order then token order
-            const uint32_t ng = __popc(gt);
-            uint32_t incl = ng;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o2;
-            }
-            uint32_t pos = n_w + incl - ng;
-            n_w += __shfl_sync(0xffffffffu, incl, 31);
-            for (uint32_t mm = gt; mm; mm &= mm - 1, ++pos) {
-                const int t = t0 + p0 + __ffs(mm) - 1;
-                if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
-                prefetch_l2(crow + t);
-                prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
-                if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+                for (uint32_t mm = gt; mm; mm &= mm - 1, ++pos) {
+                    const int t = t0 + p0 + __ffs(mm) - 1;
+                    if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
+                    prefetch_l2(crow + t);
+                    prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
+                    if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+                }
             }
             for (uint32_t mm = eq; mm; mm &= mm - 1) {
                 const uint32_t slot = atomicAdd(&sh.sc[8], 1u);
-                if (slot < kFPend) pend[slot] = static_cast<uint32_t>(p0 + __ffs(mm) - 1);
+                const int p = p0 + __ffs(mm) - 1;
+                if (slot < kFPend) pend[slot] = static_cast<uint32_t>(p);
+                prefetch_l2(crow + t0 + p);            // re-read below
             }
         }
         if (lane == 0) sh.wcnt[warp] = n_w;
@@ -792,27 +803,18 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
             const bool ranked = ncand <= kFRankMax;
             for (int i = tid; i < kFMaxChunk / 32; i += kFT) sh.u.sel.winbits[i] = 0;
             if (ranked) {
-                if (tid < ncand) {
-                    sh.u.sel.ckey[tid] = c0.x;
-                    sh.u.sel.cidx[tid] = static_cast<int32_t>(c0.y);
-                }
-                if (tid + kFT < ncand) {
-                    sh.u.sel.ckey[tid + kFT] = c1.x;
-                    sh.u.sel.cidx[tid + kFT] = static_cast<int32_t>(c1.y);
-                }
+                if (tid < ncand) sh.u.sel.ck[tid] = (static_cast<unsigned long long>(c0.x) << 32) | ~c0.y;
+                if (tid + kFT < ncand) sh.u.sel.ck[tid + kFT] = (static_cast<unsigned long long>(c1.x) << 32) | ~c1.y;
             }
             __syncthreads();
             if (ranked) {
                 for (int e = tid; e < ncand; e += kFT) {
-                    const uint32_t ke = sh.u.sel.ckey[e], ie = static_cast<uint32_t>(sh.u.sel.cidx[e]);
+                    const unsigned long long me = sh.u.sel.ck[e];
                     uint32_t rank = 0;
-#pragma unroll 4
-                    for (int f = 0; f < ncand; ++f) {
-                        const uint32_t kf = sh.u.sel.ckey[f];
-                        rank += (kf > ke) || (kf == ke && static_cast<uint32_t>(sh.u.sel.cidx[f]) < ie);
-                    }
+#pragma unroll 8
+                    for (int f = 0; f < ncand; ++f) rank += sh.u.sel.ck[f] > me ? 1u : 0u;
                     if (rank < need) {
-                        const int rel = static_cast<int>(ie) - t0;
+                        const int rel = static_cast<int>(~static_cast<uint32_t>(me)) - t0;
                         if (rel >= 0 && rel < a.chunk) atomicOr(&sh.u.sel.winbits[rel >> 5], 1u << (rel & 31));
                         else if (rel < 0) ++win_before;
                     }
@@ -984,7 +986,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         }
     }
 
-    // merge the warps' softmax states into this CTA's partial (m, l, o)
+    // merge the warps' softmax states into this CTA's partial (m, l, o);
+    // red aliases the value-staging buffers, so every warp must be done first
+    __syncthreads();
     if (lane == 0) {
 #pragma unroll
         for (int g = 0; g < GM; ++g) {

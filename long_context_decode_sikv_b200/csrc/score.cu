@@ -35,7 +35,11 @@ score_kernel(const void *__restrict__ q, const uint8_t *__restrict__ codes,
     const int t_begin = blockIdx.x * kScoreChunk;
     if (t_begin >= n_tok) return;
     const int t_end = min(t_begin + kScoreChunk, n_tok);
-    stage_table_inputs<DT>(qs, cbs, mus, q, codebook, mu, b, h, hq, group, seg);
+    {
+        TableInputs<DT> in;
+        in.load(q, codebook, mu, b, h, hq, group, seg);
+        in.store(qs, cbs, mus, group);
+    }
     __syncthreads();
     build_score_tables(sh, qs, cbs, mus, group);
 

@@ -35,26 +35,50 @@ struct ScoreTables {
     float pad[3];
 };
 
-// Loads the inputs of the tables of segment (b, h) into shared memory with one
-// round trip: the group's query rows (as fp32, `qs`, `group` x 128), the
-// segment's codebook (`cbs`, 512 float4) and channel means (`mus`, 128).
 constexpr int kTableThreads = 256;      // CTA size of every kernel that builds the tables
 
+// One thread's share of the inputs of the tables of segment (b, h): the
+// group's query rows (as fp32), the segment's codebook (512 float4) and its
+// channel means (128).  load() issues every global load at once; store()
+// writes them to shared memory (qs: group x 128, cbs, mus), so that other
+// work can be issued in between.
 template <int DT>
-__device__ __forceinline__ void stage_table_inputs(float *qs, float4 *cbs, float *mus, const void *__restrict__ q,
-                                                   const float *__restrict__ codebook, const float *__restrict__ mu,
-                                                   int b, int h, int hq, int group, int seg) {
-    constexpr int EB = ElemBytes<DT>::value;
-    constexpr int nt = kTableThreads;
-    const int tid = threadIdx.x;
-    const char *qrow = static_cast<const char *>(q) +
-                       (static_cast<size_t>(b) * hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
-#pragma unroll 1
-    for (int e = tid; e < group * kHeadDim; e += nt) qs[e] = load1<DT>(qrow, e);
-    const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
-    for (int e = tid; e < kSubspaces * kClusters; e += nt) cbs[e] = __ldg(cb + e);
-    for (int e = tid; e < kHeadDim; e += nt) mus[e] = __ldg(mu + static_cast<size_t>(seg) * kHeadDim + e);
-}
+struct TableInputs {
+    static constexpr int kQ = kMaxGroup * kHeadDim / kTableThreads;             // 4
+    static constexpr int kCb = kSubspaces * kClusters / kTableThreads;          // 2
+    float qv[kQ];
+    float4 cv[kCb];
+    float mv;
+
+    __device__ __forceinline__ void load(const void *__restrict__ q, const float *__restrict__ codebook,
+                                         const float *__restrict__ mu, int b, int h, int hq, int group, int seg) {
+        constexpr int EB = ElemBytes<DT>::value;
+        const int tid = threadIdx.x;
+        const char *qrow = static_cast<const char *>(q) +
+                           (static_cast<size_t>(b) * hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+            const int e = tid + kTableThreads * i;
+            qv[i] = (e < group * kHeadDim) ? load1<DT>(qrow, e) : 0.f;
+        }
+        const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
+#pragma unroll
+        for (int i = 0; i < kCb; ++i) cv[i] = __ldg(cb + tid + kTableThreads * i);
+        mv = (tid < kHeadDim) ? __ldg(mu + static_cast<size_t>(seg) * kHeadDim + tid) : 0.f;
+    }
+
+    __device__ __forceinline__ void store(float *qs, float4 *cbs, float *mus, int group) const {
+        const int tid = threadIdx.x;
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+            const int e = tid + kTableThreads * i;
+            if (e < group * kHeadDim) qs[e] = qv[i];
+        }
+#pragma unroll
+        for (int i = 0; i < kCb; ++i) cbs[tid + kTableThreads * i] = cv[i];
+        if (tid < kHeadDim) mus[tid] = mv;
+    }
+};
 
 // Builds q_bar, LUT, q_bar.mu and T2 from staged inputs with the whole CTA.
 // Expects the staged inputs to be visible (a __syncthreads() after staging);
