@@ -637,45 +637,51 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         bstar = static_cast<int>(sh.sc[0]);
         above_bstar = sh.sc[1];
         const uint32_t b2 = static_cast<uint32_t>(bstar + 1) * 0x10001u;
-        // warp w scans rows w, w + 8, ... of 256 entries (8 per lane) and lists
-        // its tokens in ascending order; list positions come from one ballot
-        // per entry slot, not from a shuffle scan
-        const uint32_t below = (1u << lane) - 1u;
-        uint32_t n_w = 0;
+        // warp w scans rows w, w + 8, ... (at most 8) of 256 entries, 8 per
+        // lane: it flags the tokens above b* and keeps, per lane, a 64-bit mask
+        // of them (bit 8 r + j: entry j of the lane's r-th row) and of the
+        // tokens in b*.  One pass over the masks then lists them: lane by
+        // lane, row by row (a fixed order), positions from 7 ballots.
+        unsigned long long gmask = 0ull, emask = 0ull;
 #pragma unroll 1
-        for (int row = warp; row < nrows; row += kFW) {
+        for (int r = 0, row = warp; row < nrows; ++r, row += kFW) {
             const int p0 = row * kFRow + 8 * lane;
             uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
             const uint32_t gx = half_gt(w.x, b2), gy = half_gt(w.y, b2), gz = half_gt(w.z, b2), gw = half_gt(w.w, b2);
-            const uint32_t gt = mask8(gx, gy, gz, gw);
-            const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
-            uint32_t pos = n_w;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t bj = __ballot_sync(0xffffffffu, (gt >> j) & 1u);
-                pos += __popc(bj & below);
-                n_w += __popc(bj);
-            }
-            if (gt) {
+            const uint32_t ex = half_eq(w.x, b2), ey = half_eq(w.y, b2), ez = half_eq(w.z, b2), ew = half_eq(w.w, b2);
+            if (gx | gy | gz | gw) {
                 w.x |= gx & kSure;
                 w.y |= gy & kSure;
                 w.z |= gz & kSure;
                 w.w |= gw & kSure;
                 *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
-                for (uint32_t mm = gt; mm; mm &= mm - 1, ++pos) {
-                    const int t = t0 + p0 + __ffs(mm) - 1;
-                    if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
-                    prefetch_l2(crow + t);
-                    prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
-                    if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
-                }
+                gmask |= static_cast<unsigned long long>(mask8(gx, gy, gz, gw)) << (8 * r);
             }
-            for (uint32_t mm = eq; mm; mm &= mm - 1) {
-                const uint32_t slot = atomicAdd(&sh.sc[8], 1u);
-                const int p = p0 + __ffs(mm) - 1;
-                if (slot < kFPend) pend[slot] = static_cast<uint32_t>(p);
-                prefetch_l2(crow + t0 + p);            // re-read below
-            }
+            if (ex | ey | ez | ew) emask |= static_cast<unsigned long long>(mask8(ex, ey, ez, ew)) << (8 * r);
+        }
+        const uint32_t below = (1u << lane) - 1u;
+        const uint32_t cnt = __popcll(gmask);
+        uint32_t pos = 0, n_w = 0;
+#pragma unroll
+        for (int bit = 0; bit < 7; ++bit) {
+            const uint32_t bb = __ballot_sync(0xffffffffu, (cnt >> bit) & 1u);
+            pos += static_cast<uint32_t>(__popc(bb & below)) << bit;
+            n_w += static_cast<uint32_t>(__popc(bb)) << bit;
+        }
+        for (unsigned long long mm = gmask; mm; mm &= mm - 1, ++pos) {
+            const int bit = __ffsll(static_cast<long long>(mm)) - 1;
+            const int t = t0 + (warp + kFW * (bit >> 3)) * kFRow + 8 * lane + (bit & 7);
+            if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
+            prefetch_l2(crow + t);
+            prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
+            if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+        }
+        for (unsigned long long mm = emask; mm; mm &= mm - 1) {
+            const int bit = __ffsll(static_cast<long long>(mm)) - 1;
+            const int p = (warp + kFW * (bit >> 3)) * kFRow + 8 * lane + (bit & 7);
+            const uint32_t slot = atomicAdd(&sh.sc[8], 1u);
+            if (slot < kFPend) pend[slot] = static_cast<uint32_t>(p);
+            prefetch_l2(crow + t0 + p);            // re-read below
         }
         if (lane == 0) sh.wcnt[warp] = n_w;
         __syncthreads();
