@@ -46,7 +46,7 @@ constexpr int kFListCap = 2048;          // attended tokens staged per window
 constexpr int kFMaxNpt = 64;             // token slots per thread at most
 constexpr int kFMaxChunk = kFMaxNpt * kFT;
 constexpr int kFRankMax = 512;           // up to this many candidates: rank directly
-constexpr int kFUnroll = 8;              // code rows in flight per thread
+constexpr int kFUnroll = 4;              // code rows in flight per thread
 constexpr int kFPrefetchRows = 16;       // code rows per thread sent to L2 during the prologue
 constexpr int kFPend = kFBins / 4;       // threshold-bin tokens of a CTA re-scored together
 constexpr int kFDirect = kFBins / 2;     // attended tokens listed directly during the scans
@@ -373,16 +373,18 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 
-// Waits for this thread's outstanding cp.async copies.
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
+// Closes the current group of this thread's cp.async copies.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
-// Value rows staged per round by a warp.
+// Waits until at most one group of this thread's copies is still in flight.
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Value rows staged by a warp: two halves of its buffer, so that one half
+// is consumed while the other is in flight.
 template <int DT>
 struct VStage {
     static constexpr int kRowBytes = kHeadDim * ElemBytes<DT>::value;
-    static constexpr int kRows = kFVBytes / kRowBytes;      // 16 (bf16) or 8 (fp32)
+    static constexpr int kHalf = kFVBytes / kRowBytes / 2;  // 8 (bf16) or 4 (fp32) rows
 };
 
 // Starts copying the value rows of tokens tok[j0 .. j0 + n) into vb (row j
@@ -544,28 +546,24 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     // ---- scores of this chunk -> histogram and per-slot bins
     {
         float *so = a.scores_out ? a.scores_out + kv_seg : nullptr;
-        // rows of the next group are requested before the current group is
-        // scored, so each thread always has a group of rows in flight
-        uint4 nxt[kFUnroll];
+        // Two register groups of kFUnroll rows per thread, ping-ponged: one is
+        // scored while the other is in flight.  Loads are guarded only by the
+        // warp-uniform slot count; their token index is clamped into the cache
+        // (rows of sinks or past the sequence are loaded and discarded).
+        const int tmax = a.nmax - 1;
+        uint4 ra[kFUnroll], rb[kFUnroll];
 #pragma unroll
-        for (int u = 0; u < kFUnroll; ++u) {
-            const int t = t0 + kFT * u + my;
-            nxt[u] = (u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll 1
-        for (int i0 = 0; i0 < npt; i0 += kFUnroll) {
-            uint4 rows[kFUnroll];
+        for (int u = 0; u < kFUnroll; ++u) ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
+        auto load_group = [&](uint4 (&r)[kFUnroll], int i0) {
 #pragma unroll
-            for (int u = 0; u < kFUnroll; ++u) rows[u] = nxt[u];
-#pragma unroll
-            for (int u = 0; u < kFUnroll; ++u) {
-                const int t = t0 + kFT * (i0 + kFUnroll + u) + my;
-                nxt[u] = (i0 + kFUnroll + u < npt && t >= tstart && t < t1) ? __ldcs(crow + t) : make_uint4(0, 0, 0, 0);
-            }
+            for (int u = 0; u < kFUnroll; ++u)
+                if (i0 + u < npt) r[u] = __ldcs(crow + min(t0 + kFT * (i0 + u) + my, tmax));
+        };
+        auto score_group = [&](const uint4 (&r)[kFUnroll], int i0) {
             float sc2[kFUnroll];
 #pragma unroll
             for (int u = 0; u < kFUnroll; u += 2) {
-                const float2 v = lut2_score2(sh.u.tab.t2, rows[u], rows[u + 1], lane, qmu);
+                const float2 v = lut2_score2(sh.u.tab.t2, r[u], r[u + 1], lane, qmu);
                 sc2[u] = v.x;
                 sc2[u + 1] = v.y;
             }
@@ -574,19 +572,29 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                 const int i = i0 + u;
                 if (i >= npt) break;
                 const int t = t0 + kFT * i + my;
-                uint16_t e = 0;
+                uint32_t e = 0;
                 if (t >= tstart && t < t1) {
                     const float sv = sc2[u];
-                    int bi = 0;
-                    if (!bin_flat) bi = min(max(__float2int_rz((sv - bin_lo) * bin_inv), 0), kFBins - 1);
+                    // sv >= bin_lo up to rounding; a negative product converts to 0
+                    const uint32_t bi = bin_flat ? 0u : min(__float2uint_rz((sv - bin_lo) * bin_inv),
+                                                            static_cast<uint32_t>(kFBins - 1));
                     atomicAdd(&sh.hist[bi], 1u);
-                    e = static_cast<uint16_t>(bi + 1);
+                    e = bi + 1u;
                     if (so) so[t] = sv;
                 } else if (so && t < t1) {
                     so[t] = -INFINITY;
                 }
-                sh.bins[i * kFT + tid] = e;
+                sh.bins[i * kFT + tid] = static_cast<uint16_t>(e);
             }
+        };
+        load_group(ra, 0);
+#pragma unroll 1
+        for (int i0 = 0; i0 < npt; i0 += 2 * kFUnroll) {
+            load_group(rb, i0 + kFUnroll);
+            score_group(ra, i0);
+            if (i0 + kFUnroll >= npt) break;
+            load_group(ra, i0 + 2 * kFUnroll);
+            score_group(rb, i0 + kFUnroll);
         }
     }
     __syncthreads();
@@ -914,9 +922,15 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                 char *vb = sh.u.at.vbuf[warp];
                 tok[lane] = t;
                 __syncwarp();
-                // the first value rows are in flight while the logits are formed
-                constexpr int kVR = VStage<DT>::kRows;
-                warp_stage_v<DT>(vb, tok, 0, min(nb, kVR), vseg, lane);
+                // the first value rows are in flight while the logits are formed;
+                // then each half-buffer is refilled as soon as it is consumed
+                // (one copy group per half, so waiting for "all but one group"
+                // always means the half about to be read)
+                constexpr int kVH = VStage<DT>::kHalf, kHB = kVH * VStage<DT>::kRowBytes;
+                warp_stage_v<DT>(vb, tok, 0, min(nb, kVH), vseg, lane);
+                cp_async_commit();
+                warp_stage_v<DT>(vb + kHB, tok, kVH, max(0, min(nb - kVH, kVH)), vseg, lane);
+                cp_async_commit();
                 float lg[GM];
 #pragma unroll
                 for (int g = 0; g < GM; ++g) lg[g] = -INFINITY;
@@ -943,15 +957,14 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                 }
                 warp_softmax_batch(ws, lg);
 #pragma unroll 1
-                for (int j0 = 0; j0 < nb; j0 += kVR) {
-                    const int n = min(kVR, nb - j0);
-                    if (j0 > 0) {
-                        __syncwarp();          // every lane is done with the previous rows
-                        warp_stage_v<DT>(vb, tok, j0, n, vseg, lane);
-                    }
-                    cp_async_wait_all();
+                for (int j0 = 0, half = 0; j0 < nb; j0 += kVH, half ^= 1) {
+                    char *hb = vb + half * kHB;
+                    cp_async_wait_one();
                     __syncwarp();
-                    warp_fma_v<DT, GM>(ws, vb, lg, j0, n, lane);
+                    warp_fma_v<DT, GM>(ws, hb, lg, j0, min(kVH, nb - j0), lane);
+                    __syncwarp();              // every lane is done with this half
+                    warp_stage_v<DT>(hb, tok, j0 + 2 * kVH, max(0, min(nb - j0 - 2 * kVH, kVH)), vseg, lane);
+                    cp_async_commit();
                 }
                 __syncwarp();                  // tok and vbuf are reused by the next batch
             }
