@@ -539,8 +539,8 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         }
     }
     __syncthreads();
-    const float bin_lo = sh.bin_lo, bin_inv = sh.bin_inv;
-    const bool bin_flat = sh.bin_flat != 0;
+    const float bin_mul = sh.bin_flat ? 0.f : sh.bin_inv;
+    const float bin_add = sh.bin_flat ? 0.f : -sh.bin_lo * sh.bin_inv;
     const float qmu = sh.u.tab.qmu;
 
     // ---- scores of this chunk -> histogram and per-slot bins
@@ -551,6 +551,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         // warp-uniform slot count; their token index is clamped into the cache
         // (rows of sinks or past the sequence are loaded and discarded).
         const int tmax = a.nmax - 1;
+        const uint32_t span = static_cast<uint32_t>(max(t1 - tstart, 0));   // scored tokens of the chunk
         uint4 ra[kFUnroll], rb[kFUnroll];
 #pragma unroll
         for (int u = 0; u < kFUnroll; ++u) ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -573,11 +574,11 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                 if (i >= npt) break;
                 const int t = t0 + kFT * i + my;
                 uint32_t e = 0;
-                if (t >= tstart && t < t1) {
+                if (static_cast<uint32_t>(t - tstart) < span) {
                     const float sv = sc2[u];
-                    // sv >= bin_lo up to rounding; a negative product converts to 0
-                    const uint32_t bi = bin_flat ? 0u : min(__float2uint_rz((sv - bin_lo) * bin_inv),
-                                                            static_cast<uint32_t>(kFBins - 1));
+                    // sv >= the lowest possible score up to rounding; a negative
+                    // value converts to 0
+                    const uint32_t bi = min(__float2uint_rz(fmaf(sv, bin_mul, bin_add)), static_cast<uint32_t>(kFBins - 1));
                     atomicAdd(&sh.hist[bi], 1u);
                     e = bi + 1u;
                     if (so) so[t] = sv;
