@@ -124,6 +124,7 @@ SIKV_API size_t sikv_score_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_topk_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_sparse_attn_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_decode_host_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
  * (0 on bad params). */
@@ -202,6 +203,28 @@ SIKV_API sikv_status sikv_decode(const sikv_params *p, const void *q, const void
                         const int32_t *seq_lens, const int32_t *k_per_seq, void *out,
                         int32_t *idx_out, float *scores_out, void *workspace,
                         size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * sikv_decode_host -- sikv_decode with the query and the output in host
+ * memory: q_host and out_host are [B][Hq][D] in the cache dtype.  Page-locked
+ * buffers (cudaHostAlloc, cudaHostRegister) are device-addressable, so the
+ * decode kernels read the query and write the output in place over the host
+ * link; pageable buffers are staged through the workspace with
+ * cudaMemcpyAsync (then the copies synchronize with the host).  Everything is
+ * enqueued on `stream`; returns once enqueued, and out_host is valid after
+ * the stream is synchronized.  K,
+ * V, codes, codebook, mu, seq_lens and k_per_seq are device pointers as for
+ * sikv_decode.  The workspace is sikv_decode_host_workspace_size() bytes:
+ * the decode workspace followed by device copies of q and of the output.
+ * Null host pointers return SIKV_ERR_INVALID_ARG; a failed copy returns
+ * SIKV_ERR_CUDA.  The paper has no counterpart: this is the host-facing form
+ * of the decode step [SIKV 2.1.2-2.1.4], one call per step for a caller
+ * that keeps queries and outputs on the host.
+ */
+SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const void *K, const void *V,
+                                      const uint8_t *codes, const float *codebook, const float *mu,
+                                      const int32_t *seq_lens, const int32_t *k_per_seq, void *out_host,
+                                      void *workspace, size_t workspace_bytes, sikv_stream_t stream);
 
 /*
  * sikv_sparse_attn_static -- sikv_sparse_attn for callers that cannot

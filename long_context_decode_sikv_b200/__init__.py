@@ -16,9 +16,9 @@ import numpy as np
 import torch
 
 from ._binding import (EXPORTED, SIKV_DEVERR_INDEX, SIKV_DEVERR_SEQ_LEN, SIKV_DEVERR_TOPK,  # noqa: F401
-                       SIKV_DTYPE_BF16, SIKV_DTYPE_F32, Params, SikvError, Workspace, default_scale, lib,
-                       library_path, make_params, sikv_decode, sikv_encode_keys, sikv_score,
-                       sikv_sparse_attn, sikv_topk, version, workspace_size)
+                       SIKV_DTYPE_BF16, SIKV_DTYPE_F32, DecodeHostPlan, Params, SikvError, Workspace,
+                       default_scale, lib, library_path, make_params, sikv_decode, sikv_decode_host,
+                       sikv_encode_keys, sikv_score, sikv_sparse_attn, sikv_topk, version, workspace_size)
 
 
 def to_device(a: np.ndarray, dtype: str, device) -> torch.Tensor:

@@ -33,7 +33,7 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
             "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
-            "sikv_sparse_attn_static")
+            "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host")
 
 
 class SikvError(RuntimeError):
@@ -95,7 +95,8 @@ def lib() -> ctypes.CDLL:
         L.sikv_workspace_init.argtypes = [vp, sz, vp]
         L.sikv_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(i32)]
         for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
-                  "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size"):
+                  "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size",
+                  "sikv_decode_host_workspace_size"):
             getattr(L, n).restype = sz
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
@@ -105,8 +106,9 @@ def lib() -> ctypes.CDLL:
         L.sikv_topk.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_sparse_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_decode_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
-                  "sikv_topk", "sikv_sparse_attn", "sikv_decode"):
+                  "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -138,6 +140,20 @@ def _ptr(t, name, dtype=None, shape=None, device=None, optional=False):
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor; pin it for asynchronous copies")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
@@ -271,3 +287,62 @@ def sikv_decode(p: Params, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, ou
 
 def default_scale(head_dim: int = 128) -> float:
     return 1.0 / math.sqrt(head_dim)
+
+
+def _decode_device_args(p: Params, K, V, codes, codebook, mu, seq_lens, k_per_seq):
+    dev = K.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    return dev, (_ptr(K, "K", p.torch_dtype, (B, H, N, D), dev), _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev),
+                 _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+                 _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+                 _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+                 _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev))
+
+
+def sikv_decode_host(p: Params, q_host, K, V, codes, codebook, mu, seq_lens, k_per_seq, out_host,
+                     workspace=None, stream=None):
+    """One decode step with q and out in host memory (CPU tensors [B][Hq][D]).
+
+    Returns after enqueueing the upload, the step and the download on
+    ``stream``; synchronize before reading ``out_host``.
+    """
+    dev, dargs = _decode_device_args(p, K, V, codes, codebook, mu, seq_lens, k_per_seq)
+    shape = (p.batch, p.num_q_heads, p.head_dim)
+    q = _host_ptr(q_host, "q_host", p.torch_dtype, shape)
+    o = _host_ptr(out_host, "out_host", p.torch_dtype, shape)
+    ws = _ws("decode_host", p, workspace, dev, stream)
+    _check(lib().sikv_decode_host(ctypes.byref(p), q, *dargs, o, ws.ptr, ws.nbytes, _stream(stream, dev)),
+           "sikv_decode_host")
+    return ws
+
+
+class DecodeHostPlan:
+    """sikv_decode_host with the device-side arguments checked once.
+
+    A serving loop that keeps queries and outputs on the host builds one plan
+    per cache and calls it once per step with the step's host buffers (pinned
+    CPU tensors of shape [B][Hq][D] and the cache's dtype); each call is one
+    C call that enqueues the upload, the decode step and the download.
+    """
+
+    def __init__(self, p: Params, K, V, codes, codebook, mu, seq_lens, k_per_seq, workspace=None, stream=None):
+        self.p = p
+        dev, self._dargs = _decode_device_args(p, K, V, codes, codebook, mu, seq_lens, k_per_seq)
+        self._keep = (K, V, codes, codebook, mu, seq_lens, k_per_seq)
+        self.workspace = _ws("decode_host", p, workspace, dev, stream)
+        self._shape = (p.batch, p.num_q_heads, p.head_dim)
+        self._dtype = p.torch_dtype
+        self._stream = _stream(stream, dev)
+        self._pref = ctypes.byref(p)
+        self._fn = lib().sikv_decode_host
+
+    def __call__(self, q_host, out_host):
+        if q_host.is_cuda or out_host.is_cuda or q_host.dtype != self._dtype or out_host.dtype != self._dtype \
+                or q_host.shape != self._shape or out_host.shape != self._shape \
+                or not (q_host.is_contiguous() and out_host.is_contiguous()):
+            _host_ptr(q_host, "q_host", self._dtype, self._shape)       # raises with the reason
+            _host_ptr(out_host, "out_host", self._dtype, self._shape)
+        st = self._fn(self._pref, q_host.data_ptr(), *self._dargs, out_host.data_ptr(), self.workspace.ptr,
+                      self.workspace.nbytes, self._stream)
+        if st != 0:
+            raise SikvError(st, "sikv_decode_host")

@@ -77,10 +77,71 @@ DecodeLayout decode_layout(const sikv_params &p) {
 }
 
 int device_sm_count() {
+    static int cached[64];                     // per device, 0 until first asked
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
     return n;
+}
+
+// Workspace of sikv_decode_host: the decode workspace, then the device copies
+// of the query and of the output.
+struct HostLayout {
+    size_t bytes = 0, q = 0, out = 0, total = 0;   // bytes: one query (= one output) tensor
+};
+
+HostLayout host_layout(const sikv_params &p, size_t decode_total) {
+    HostLayout H;
+    const size_t eb = p.dtype == SIKV_DTYPE_F32 ? 4 : 2;
+    H.bytes = static_cast<size_t>(p.batch) * p.num_q_heads * p.head_dim * eb;
+    H.q = align_up(decode_total, 256);
+    H.out = align_up(H.q + H.bytes, 256);
+    H.total = align_up(H.out + H.bytes, 256);
+    return H;
+}
+
+// The device address of a page-locked host buffer, or null for pageable
+// memory (which then goes through a staged copy).
+void *device_view(const void *host) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (at.type != cudaMemoryTypeHost || !at.devicePointer) return nullptr;
+    return at.devicePointer;
+}
+
+// One decode step on device buffers (arguments checked here, except q and
+// out, which the callers check).
+sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, const void *V, const uint8_t *codes,
+                        const float *codebook, const float *mu, const int32_t *seq_lens, const int32_t *k_per_seq,
+                        void *out, int32_t *idx_out, float *scores_out, void *workspace, size_t workspace_bytes,
+                        cudaStream_t s) {
+    const sikv_params *p = &pp;
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR(V);
+    SIKV_REQUIRE_PTR(codes);
+    SIKV_REQUIRE_PTR(codebook);
+    SIKV_REQUIRE_PTR(mu);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR4(k_per_seq);
+    const DecodeLayout L = decode_layout(*p);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
+    char *ws = static_cast<char *>(workspace);
+    int32_t *status = reinterpret_cast<int32_t *>(ws);
+    const FusedPlan plan = fused_plan(*p);
+    if (plan.ok)
+        return launch_decode_fused(*p, plan, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
+                                   scores_out, ws, L.fused, status, s);
+    float *sc = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores);
+    int32_t *ix = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
+    SIKV_TRY(launch_score(*p, q, codes, codebook, mu, seq_lens, sc, status, s));
+    if (p->max_topk > 0) SIKV_TRY(launch_topk(*p, sc, seq_lens, k_per_seq, ix, status, s));
+    return launch_sparse_attn(*p, q, K, V, codes, codebook, mu, ix, k_per_seq, seq_lens, out, ws, L.attn,
+                              status, s);
 }
 
 }  // namespace sikv
@@ -143,6 +204,11 @@ size_t sikv_sparse_attn_workspace_size(const sikv_params *p) {
 size_t sikv_decode_workspace_size(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
     return decode_layout(*p).total;
+}
+
+size_t sikv_decode_host_workspace_size(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return sikv::host_layout(*p, decode_layout(*p).total).total;
 }
 
 int32_t sikv_decode_launches(const sikv_params *p) {
@@ -222,31 +288,40 @@ sikv_status sikv_decode(const sikv_params *p, const void *q, const void *K, cons
                         float *scores_out, void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
     SIKV_TRY(check_params(p));
     SIKV_REQUIRE_PTR(q);
-    SIKV_REQUIRE_PTR(K);
-    SIKV_REQUIRE_PTR(V);
-    SIKV_REQUIRE_PTR(codes);
-    SIKV_REQUIRE_PTR(codebook);
-    SIKV_REQUIRE_PTR(mu);
-    SIKV_REQUIRE_PTR4(seq_lens);
-    SIKV_REQUIRE_PTR4(k_per_seq);
     SIKV_REQUIRE_PTR(out);
     if (idx_out) SIKV_REQUIRE_PTR4(idx_out);
     if (scores_out) SIKV_REQUIRE_PTR4(scores_out);
-    const DecodeLayout L = decode_layout(*p);
-    SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
+    return sikv::decode_step(*p, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out, scores_out,
+                             workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const void *K, const void *V,
+                             const uint8_t *codes, const float *codebook, const float *mu,
+                             const int32_t *seq_lens, const int32_t *k_per_seq, void *out_host,
+                             void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    if (!q_host || !out_host) return SIKV_ERR_INVALID_ARG;
+    const size_t decode_total = decode_layout(*p).total;
+    const sikv::HostLayout H = sikv::host_layout(*p, decode_total);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, H.total));
     char *ws = static_cast<char *>(workspace);
-    int32_t *status = reinterpret_cast<int32_t *>(ws);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const FusedPlan plan = fused_plan(*p);
-    if (plan.ok)
-        return launch_decode_fused(*p, plan, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
-                                   scores_out, ws, L.fused, status, s);
-    float *sc = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores);
-    int32_t *ix = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
-    SIKV_TRY(launch_score(*p, q, codes, codebook, mu, seq_lens, sc, status, s));
-    if (p->max_topk > 0) SIKV_TRY(launch_topk(*p, sc, seq_lens, k_per_seq, ix, status, s));
-    return launch_sparse_attn(*p, q, K, V, codes, codebook, mu, ix, k_per_seq, seq_lens, out, ws, L.attn,
-                              status, s);
+    // page-locked host buffers are device-addressable (unified addressing):
+    // the kernels then read the query and write the output in place, over the
+    // host link, with no staging copy; pageable buffers are staged in the
+    // workspace with cudaMemcpyAsync
+    const void *q_dev = sikv::device_view(q_host);
+    void *out_dev = sikv::device_view(out_host);
+    if (!q_dev) {
+        if (cudaMemcpyAsync(ws + H.q, q_host, H.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return SIKV_ERR_CUDA;
+        q_dev = ws + H.q;
+    }
+    SIKV_TRY(sikv::decode_step(*p, q_dev, K, V, codes, codebook, mu, seq_lens, k_per_seq,
+                               out_dev ? out_dev : ws + H.out, nullptr, nullptr, workspace, decode_total, s));
+    if (!out_dev &&
+        cudaMemcpyAsync(out_host, ws + H.out, H.bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SIKV_ERR_CUDA;
+    return SIKV_OK;
 }
 
 }  // extern "C"

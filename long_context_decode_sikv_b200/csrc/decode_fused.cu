@@ -1115,9 +1115,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
 template <int DT, int GM>
 sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStream_t stream) {
     auto kern = decode_fused_kernel<DT, GM>;
-    const size_t smem = sizeof(FusedSmem<GM>);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return SIKV_ERR_CUDA;
+    const size_t smem = sizeof(FusedSmem<GM>);   // limit raised by fused_plan on this device
     FusedArgs a = args;
     void *params[] = {&a};
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(plan.grid),
@@ -1125,8 +1123,17 @@ sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStr
     return e == cudaSuccess ? SIKV_OK : SIKV_ERR_CUDA;
 }
 
+// Per device: the kernel's dynamic shared-memory limit is raised once, and
+// its occupancy (CTAs per SM) is computed once.  Values are idempotent, so
+// concurrent first calls only repeat the same work.
+constexpr int kMaxDevices = 64;
+
 template <int DT, int GM>
 int occupancy_of() {
+    static int cached[kMaxDevices];            // 0: unknown, else occupancy + 1
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev] - 1;
     // the occupancy calculator honours the kernel's dynamic shared-memory
     // limit, which must be raised above the 48 KB default first
     auto kern = decode_fused_kernel<DT, GM>;
@@ -1136,6 +1143,7 @@ int occupancy_of() {
     int blocks = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kFT, sizeof(FusedSmem<GM>)) != cudaSuccess)
         return 0;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev] = blocks + 1;
     return blocks;
 }
 

@@ -96,3 +96,36 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         sk.sikv_topk(p, torch.zeros(2, 2, 4096), torch.zeros(2, dtype=torch.int32),
                      torch.zeros(2, dtype=torch.int32), torch.zeros(2, 2, 256, dtype=torch.int32))
+
+
+def test_decode_host_validates_without_launch():
+    """sikv_decode_host: its workspace holds the decode workspace plus device
+    copies of q and out; null host buffers are refused before any copy."""
+    p = _p()
+    L = sk.lib()
+    n_dec = L.sikv_decode_workspace_size(ctypes.byref(p))
+    n_host = L.sikv_decode_host_workspace_size(ctypes.byref(p))
+    q_bytes = p.batch * p.num_q_heads * p.head_dim * 2
+    assert n_host >= n_dec + 2 * q_bytes
+    bad = sk.make_params("bf16", 2, 7, 2, 4096, 64, 256)
+    assert L.sikv_decode_host_workspace_size(ctypes.byref(bad)) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.sikv_decode_host(ctypes.byref(p), None, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            n_host, None)
+    assert st == 1                                       # SIKV_ERR_INVALID_ARG: q_host is null
+    st = L.sikv_decode_host(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None, fake,
+                            n_host, None)
+    assert st == 1                                       # out_host is null
+    st = L.sikv_decode_host(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            n_host, None)
+    assert st == 1                                       # invalid parameters
+
+
+def test_decode_host_binding_refuses_device_or_misshapen_buffers():
+    p = _p()
+    import torch
+    with pytest.raises((TypeError, ValueError)):
+        bnd._host_ptr(torch.zeros(2, 8, 64, dtype=torch.bfloat16), "q_host", p.torch_dtype, (2, 8, 128))
+    with pytest.raises(TypeError):
+        bnd._host_ptr(torch.zeros(2, 8, 128, dtype=torch.float32), "q_host", p.torch_dtype, (2, 8, 128))
+    assert bnd._host_ptr(torch.zeros(2, 8, 128, dtype=torch.bfloat16), "q_host", p.torch_dtype, (2, 8, 128))

@@ -105,3 +105,36 @@ def test_fused_all_scores_tied_takes_lowest_indices():
     assert np.array_equal(o_idx, np.arange(S, S + k))
     assert np.array_equal(idx[0, 0].cpu().numpy(), o_idx)
     assert np.allclose(gu.to_f64(out)[0], o_out, atol=2e-2, rtol=1e-2)
+
+
+@pytest.mark.parametrize("name", ["gqa5", "ragged-empty-chunks", "f32-one-head"])
+def test_decode_host_matches_device_decode(name):
+    """sikv_decode_host (query and output in host memory: page-locked, read
+    and written in place, or pageable, staged) and its prepared form give
+    exactly what sikv_decode gives on device buffers."""
+    dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1))
+    dw.encode()
+    c, p = dw.cache, dw.p
+    for step in (0, 1):
+        out_d = torch.empty_like(dw.q[step])
+        sk.sikv_decode(p, dw.q[step], c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, out_d).check()
+        qh = dw.q[step].cpu().pin_memory()
+        oh = torch.full(tuple(qh.shape), 7.0, dtype=qh.dtype).pin_memory()
+        ws = sk.sikv_decode_host(p, qh, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, oh)
+        torch.cuda.synchronize()
+        assert ws.check() == 0
+        assert torch.equal(oh, out_d.cpu()), (name, step)
+        # pageable host memory takes the staged-copy path
+        qp = dw.q[step].cpu()
+        op = torch.full(tuple(qp.shape), 7.0, dtype=qp.dtype)
+        assert not qp.is_pinned()
+        sk.sikv_decode_host(p, qp, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, op, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(op, out_d.cpu()), (name, step)
+        plan = sk.DecodeHostPlan(p, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k)
+        oh2 = torch.zeros_like(oh).pin_memory()
+        plan(qh, oh2)
+        plan(qh, oh2)                                   # repeated calls: same answer
+        torch.cuda.synchronize()
+        assert plan.workspace.check() == 0
+        assert torch.equal(oh2, out_d.cpu()), (name, step)
