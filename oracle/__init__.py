@@ -43,7 +43,10 @@ R10 softmax scale 1/sqrt(D);
 R11 k counts non-sink tokens only;
 R12 top-k ties go to the lower token index;
 R13 the selected set is returned in ascending token order;
-R14 a selected key is reconstructed as mu + c[s][code_s].
+R14 a selected key is reconstructed as mu + c[s][code_s];
+R19 a token appended at decode time is coded against the prefill mean, which
+    stays frozen;
+R20 the codebook stays frozen too: appended tokens do not move the centroids.
 """
 
 from __future__ import annotations
@@ -149,6 +152,21 @@ def unpack_codes(packed: np.ndarray) -> np.ndarray:
     code[:, 0::2] = packed & 0x0F
     code[:, 1::2] = packed >> 4
     return code
+
+
+def append_codes(packed: np.ndarray, K: np.ndarray, mu: np.ndarray, start: int, count: int) -> np.ndarray:
+    """Decode-time append (R19, R20): the code rows of tokens [start, start+count)
+    become the packed sign codes of their keys against the frozen prefill mean
+    [SIKV §2.1.1, §2.1.3]; every other row is kept.  Returns a new array.
+
+    The pages give the encoding of a key but say nothing of keys that arrive
+    after prefill; the plainest reading codes them like prefill keys with the
+    statistics fixed at prefill.
+    """
+    out = np.array(packed, dtype=np.uint8, copy=True)
+    if count > 0:
+        out[start:start + count] = pack_codes(sign_codes(np.asarray(K)[start:start + count], mu))
+    return out
 
 
 def codebook(K: np.ndarray, mu: np.ndarray, code: np.ndarray, num_sinks: int = DEFAULT_SINKS):

@@ -351,10 +351,58 @@ def check_needle_recall(o):
     assert set(hi.needle_pos.tolist()) <= set(idx.tolist())
 
 
+# --------------------------------------------------------------------------
+# decode-time append (R19, R20: frozen prefill mean and codebook)
+# --------------------------------------------------------------------------
+
+def check_append_by_construction(o):
+    """Appended rows carry the sign patterns their keys were built with,
+    relative to the prefill mean; the other rows are untouched.  Heavy
+    appended keys would drag a re-estimated mean far enough to flip the
+    small-margin bits, so a mean that moves with the appends is caught."""
+    rng = np.random.default_rng(19)
+    d, s, n0, n_pat, n_heavy, n_tail = 16, 8, 80, 6, 6, 4
+    K0 = rng.standard_normal((n0, d)).astype(np.float32).astype(np.float64)
+    mu = o.channel_mean(K0, s)
+    want = rng.integers(0, 16, size=(n_pat, d // 4))
+    Kp = np.empty((n_pat, d))
+    for t in range(n_pat):
+        for sub in range(d // 4):
+            for i in range(4):
+                bit = (int(want[t, sub]) >> i) & 1
+                mag = float(rng.uniform(0.01, 0.05))
+                Kp[t, 4 * sub + i] = float(mu[4 * sub + i]) + (mag if bit else -mag)
+    Kh = np.asarray(mu, dtype=np.float64)[None, :] + 50.0 * np.ones((n_heavy, d))
+    Kt = rng.standard_normal((n_tail, d))
+    K = np.concatenate([K0, Kp, Kh, Kt]).astype(np.float32).astype(np.float64)
+    before = np.zeros((K.shape[0], d // 8), dtype=np.uint8)
+    before[:n0] = o.pack_codes(o.sign_codes(K0, mu))
+    before[n0 + n_pat + n_heavy:] = 0xA5
+    got = o.append_codes(before, K, mu, n0, n_pat + n_heavy)
+    assert np.array_equal(got[:n0], before[:n0])
+    assert np.array_equal(got[n0 + n_pat + n_heavy:], before[n0 + n_pat + n_heavy:])
+    assert np.array_equal(o.unpack_codes(got[n0:n0 + n_pat]), want)
+    assert np.all(got[n0 + n_pat:n0 + n_pat + n_heavy] == 0xFF)
+    assert np.array_equal(o.append_codes(before, K, mu, n0, 0), before)
+
+
+def check_append_golden(o):
+    """Appending the hand-worked D=8 vectors reproduces their fixture codes."""
+    g = _load("sign_codes_d8.json")
+    K = np.asarray(g["keys"], dtype=np.float32).astype(np.float64)
+    mu = np.asarray(g["mu"], dtype=np.float32)
+    n = K.shape[0]
+    cache = np.full((n + 2, 1), 0x5A, dtype=np.uint8)
+    Kc = np.concatenate([K, np.zeros((2, K.shape[1]))])
+    got = o.append_codes(cache, Kc, mu, 0, n)
+    assert got[:n].tolist() == g["packed"]
+    assert got[n:].tolist() == [[0x5A], [0x5A]]
+
+
 ALL_CHECKS = [
     check_exact_sum, check_round_to_f32, check_channel_mean, check_sign_codes_golden,
     check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
     check_one_member_clusters_reconstruct, check_scores_golden, check_lut_identity,
     check_topk, check_attention_golden, check_attention_full_selection_is_dense,
-    check_attention_invariants, check_needle_recall,
+    check_attention_invariants, check_needle_recall, check_append_by_construction, check_append_golden,
 ]

@@ -80,6 +80,16 @@ def _mut_scores_no_qmu(q_group, mu, centroids, code, num_sinks=64):
     return sc, cond
 
 
+def _mut_append_reestimates_mean(packed, K, mu, start, count):
+    mu2 = oracle.channel_mean(np.asarray(K)[:start + count], 8)
+    return oracle.append_codes(packed, K, mu2, start, count)
+
+
+def _mut_append_one_row_too_many(packed, K, mu, start, count):
+    return oracle.append_codes(packed, K, mu, start, count + 1) if start + count < np.asarray(K).shape[0] \
+        else oracle.append_codes(packed, K, mu, start, count)
+
+
 MUTATIONS = {
     "strict-greater": dict(sign_codes=_mut_codes_strict),
     "msb-first-bits": dict(sign_codes=_mut_codes_msb_first),
@@ -90,6 +100,8 @@ MUTATIONS = {
     "ties-to-higher-index": dict(topk=_mut_topk_ties_high),
     "sinks-dropped": dict(sparse_attention=_mut_no_sink_keys),
     "dropped-q-dot-mu": dict(scores=_mut_scores_no_qmu),
+    "append-reestimates-mean": dict(append_codes=_mut_append_reestimates_mean),
+    "append-one-row-too-many": dict(append_codes=_mut_append_one_row_too_many),
 }
 
 
