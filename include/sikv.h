@@ -90,6 +90,7 @@ typedef enum sikv_dtype {
 #define SIKV_DEVERR_TOPK 0x2      /* k_per_seq[b] < 0, > max_topk or > max(N_b - S, 0) */
 #define SIKV_DEVERR_INDEX 0x4     /* a selected index outside [S, N_b) */
 #define SIKV_DEVERR_TIMEOUT 0x8   /* a bounded wait between the CTAs of a segment ran out */
+#define SIKV_DEVERR_APPEND 0x10   /* append rows [start_b, start_b + count_b) outside [0, max_seq_len) */
 
 typedef struct sikv_params {
     int32_t dtype;          /* sikv_dtype of K, V, q and out */
@@ -125,6 +126,7 @@ SIKV_API size_t sikv_topk_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_sparse_attn_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_host_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_append_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
  * (0 on bad params). */
@@ -190,6 +192,24 @@ SIKV_API sikv_status sikv_sparse_attn(const sikv_params *p, const void *q, const
                              const int32_t *idx, const int32_t *k_per_seq,
                              const int32_t *seq_lens, void *out, void *workspace,
                              size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * sikv_append_codes -- decode-time append [SIKV 2.1.1, 2.1.3]: the code rows
+ * of tokens [start[b], start[b] + count[b]) of every KV head of sequence b
+ * become the sign codes of those tokens' keys (already written into K by the
+ * caller) against the frozen prefill mean mu; all other rows, mu and the
+ * codebook are left unchanged.  The pages describe prefill encoding only;
+ * coding later keys against the frozen statistics is the plainest reading.
+ *  - K: device [B][Hkv][Nmax][D]; mu: device fp32 [B][Hkv][D]; codes: device
+ *    u8 [B][Hkv][Nmax][D/8], written in place.
+ *  - start, count: device int32 [B]; a sequence with start < 0, count < 0 or
+ *    start + count > Nmax sets SIKV_DEVERR_APPEND and is skipped.  The caller
+ *    raises seq_lens afterwards to make the new tokens visible to decode.
+ *  - workspace: sikv_append_workspace_size() bytes (the status header only).
+ */
+SIKV_API sikv_status sikv_append_codes(const sikv_params *p, const void *K, const int32_t *start,
+                                       const int32_t *count, const float *mu, uint8_t *codes, void *workspace,
+                                       size_t workspace_bytes, sikv_stream_t stream);
 
 /*
  * sikv_decode -- one whole decode step: sikv_score, sikv_topk and

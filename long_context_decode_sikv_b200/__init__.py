@@ -15,10 +15,11 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from ._binding import (EXPORTED, SIKV_DEVERR_INDEX, SIKV_DEVERR_SEQ_LEN, SIKV_DEVERR_TOPK,  # noqa: F401
-                       SIKV_DTYPE_BF16, SIKV_DTYPE_F32, DecodeHostPlan, Params, SikvError, Workspace,
-                       default_scale, lib, library_path, make_params, sikv_decode, sikv_decode_host,
-                       sikv_encode_keys, sikv_score, sikv_sparse_attn, sikv_topk, version, workspace_size)
+from ._binding import (EXPORTED, SIKV_DEVERR_APPEND, SIKV_DEVERR_INDEX, SIKV_DEVERR_SEQ_LEN,  # noqa: F401
+                       SIKV_DEVERR_TOPK, SIKV_DTYPE_BF16, SIKV_DTYPE_F32, DecodeHostPlan, Params, SikvError,
+                       Workspace, default_scale, lib, library_path, make_params, sikv_append_codes, sikv_decode,
+                       sikv_decode_host, sikv_encode_keys, sikv_score, sikv_sparse_attn, sikv_topk, version,
+                       workspace_size)
 
 
 def to_device(a: np.ndarray, dtype: str, device) -> torch.Tensor:
@@ -54,6 +55,13 @@ class SikvCache:
     def encode(self, stream=None):
         sikv_encode_keys(self.p, self.K, self.seq_lens, self.mu, self.codes, self.codebook, self.counts,
                          workspace=self.ws_encode, stream=stream)
+
+    def append(self, start: torch.Tensor, count: torch.Tensor, stream=None):
+        """Code the keys of tokens [start[b], start[b] + count[b]) (already
+        written into K and V) against the frozen prefill mean.  Raise
+        ``seq_lens`` afterwards to make them visible to ``decode``."""
+        sikv_append_codes(self.p, self.K, start, count, self.mu, self.codes, workspace=self.ws_encode,
+                          stream=stream)
 
     def decode(self, q, k_per_seq, out=None, idx_out=None, scores_out=None, stream=None):
         if out is None:

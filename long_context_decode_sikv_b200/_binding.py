@@ -25,6 +25,7 @@ SIKV_DEVERR_SEQ_LEN = 0x1
 SIKV_DEVERR_TOPK = 0x2
 SIKV_DEVERR_INDEX = 0x4
 SIKV_DEVERR_TIMEOUT = 0x8
+SIKV_DEVERR_APPEND = 0x10
 
 _STATUS = {0: "SIKV_OK", 1: "SIKV_ERR_INVALID_ARG", 2: "SIKV_ERR_UNSUPPORTED", 3: "SIKV_ERR_WORKSPACE",
            4: "SIKV_ERR_CUDA", 5: "SIKV_ERR_DEVICE"}
@@ -33,7 +34,8 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
             "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
-            "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host")
+            "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
+            "sikv_append_workspace_size", "sikv_append_codes")
 
 
 class SikvError(RuntimeError):
@@ -96,7 +98,7 @@ def lib() -> ctypes.CDLL:
         L.sikv_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(i32)]
         for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
                   "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size",
-                  "sikv_decode_host_workspace_size"):
+                  "sikv_decode_host_workspace_size", "sikv_append_workspace_size"):
             getattr(L, n).restype = sz
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
@@ -107,8 +109,9 @@ def lib() -> ctypes.CDLL:
         L.sikv_sparse_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_append_codes.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
-                  "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host"):
+                  "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -224,6 +227,20 @@ def sikv_encode_keys(p: Params, K, seq_lens, mu, codes, codebook, counts=None, w
             _ptr(counts, "counts", torch.int32, (B, H, D // 4, 16), dev, optional=True))
     ws = _ws("encode", p, workspace, dev, stream)
     _check(lib().sikv_encode_keys(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_encode_keys")
+    return ws
+
+
+def sikv_append_codes(p: Params, K, start, count, mu, codes, workspace=None, stream=None):
+    """Decode-time append: code rows [start[b], start[b] + count[b]) of every
+    KV head of sequence b against the frozen mean (K rows already written)."""
+    dev = K.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(K, "K", p.torch_dtype, (B, H, N, D), dev), _ptr(start, "start", torch.int32, (B,), dev),
+            _ptr(count, "count", torch.int32, (B,), dev), _ptr(mu, "mu", torch.float32, (B, H, D), dev),
+            _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev))
+    ws = _ws("append", p, workspace, dev, stream)
+    _check(lib().sikv_append_codes(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)),
+           "sikv_append_codes")
     return ws
 
 

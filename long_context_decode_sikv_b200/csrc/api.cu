@@ -206,6 +206,25 @@ size_t sikv_decode_workspace_size(const sikv_params *p) {
     return decode_layout(*p).total;
 }
 
+size_t sikv_append_workspace_size(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return kHeaderBytes;
+}
+
+sikv_status sikv_append_codes(const sikv_params *p, const void *K, const int32_t *start, const int32_t *count,
+                              const float *mu, uint8_t *codes, void *workspace, size_t workspace_bytes,
+                              sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR4(start);
+    SIKV_REQUIRE_PTR4(count);
+    SIKV_REQUIRE_PTR(mu);
+    SIKV_REQUIRE_PTR(codes);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, kHeaderBytes));
+    int32_t *status = reinterpret_cast<int32_t *>(workspace);
+    return sikv::launch_append(*p, K, start, count, mu, codes, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t sikv_decode_host_workspace_size(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
     return sikv::host_layout(*p, decode_layout(*p).total).total;

@@ -50,6 +50,8 @@ sikv_status launch_encode(const sikv_params &p, const void *K, const int32_t *se
                           uint8_t *codes, float *codebook, int32_t *counts, char *ws,
                           cudaStream_t stream);
 
+sikv_status launch_append(const sikv_params &p, const void *K, const int32_t *start, const int32_t *count,
+                          const float *mu, uint8_t *codes, int32_t *status, cudaStream_t stream);
 sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,
                          const float *codebook, const float *mu, const int32_t *seq_lens,
                          float *scores, int32_t *status, cudaStream_t stream);

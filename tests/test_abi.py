@@ -129,3 +129,14 @@ def test_decode_host_binding_refuses_device_or_misshapen_buffers():
     with pytest.raises(TypeError):
         bnd._host_ptr(torch.zeros(2, 8, 128, dtype=torch.float32), "q_host", p.torch_dtype, (2, 8, 128))
     assert bnd._host_ptr(torch.zeros(2, 8, 128, dtype=torch.bfloat16), "q_host", p.torch_dtype, (2, 8, 128))
+
+
+def test_append_validates_without_launch():
+    p = _p()
+    L = sk.lib()
+    assert L.sikv_append_workspace_size(ctypes.byref(p)) == 256
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.sikv_append_codes(ctypes.byref(p), None, fake, fake, fake, fake, fake, 256, None) == 1
+    assert L.sikv_append_codes(ctypes.byref(p), fake, None, fake, fake, fake, fake, 256, None) == 1
+    assert L.sikv_append_codes(ctypes.byref(p), fake, fake, fake, fake, None, fake, 256, None) == 1
+    assert L.sikv_append_codes(ctypes.byref(p), fake, fake, fake, fake, fake, fake, 16, None) == 3   # workspace too small
