@@ -300,6 +300,41 @@ def sparse_attention(q_group: np.ndarray, K: np.ndarray, V: np.ndarray, mu: np.n
     return p @ vals
 
 
+def dense_scores(q_group: np.ndarray, K: np.ndarray, num_sinks: int = DEFAULT_SINKS) -> np.ndarray:
+    """Comparison baseline, not the method: the full-precision score q_bar . K[t]
+    of every non-sink token (R9), -inf for sinks.  It is the dot product the
+    compressed-domain score of [SIKV §2.1.2] stands in for.  Returns float64 [N].
+    """
+    q_bar = group_query(q_group)
+    K = np.asarray(K, dtype=np.float64)
+    out = K @ q_bar
+    out[:min(num_sinks, K.shape[0])] = -np.inf
+    return out
+
+
+def dense_attention(q_group: np.ndarray, K: np.ndarray, V: np.ndarray, n_tok: int | None = None,
+                    scale: float | None = None) -> np.ndarray:
+    """Comparison baseline, not the method: softmax attention of each query
+    head over every token [0, n_tok) with its stored key and value (R10).  It
+    is the dense decode attention that [SIKV §2.1.4]'s sparse pass replaces.
+    Returns float64 [G][D] (zeros for an empty sequence).
+    """
+    q = np.asarray(q_group, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    n = K.shape[0] if n_tok is None else n_tok
+    g, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if n == 0:
+        return np.zeros((g, d))
+    logits = scale * (q @ K[:n].T)
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ V[:n]
+
+
 def decode_step(q_group, K, V, mu, centroids, code, k, num_sinks=DEFAULT_SINKS, scale=None):
     """One decode step of one (sequence, KV head): score, select, attend.
 

@@ -399,10 +399,47 @@ def check_append_golden(o):
     assert got[n:].tolist() == [[0x5A], [0x5A]]
 
 
+# --------------------------------------------------------------------------
+# comparison baselines (dense scoring and dense attention, not the method)
+# --------------------------------------------------------------------------
+
+def check_dense_scores_equal_lut_scores_when_exact(o):
+    """With one token per cluster the reconstruction is exact, so the
+    compressed-domain score equals the full dot product q_bar . k."""
+    s = 4
+    K, _ = _distinct_pattern_keys(s, seed=21)
+    rng = np.random.default_rng(22)
+    q = rng.standard_normal((3, K.shape[1]))
+    mu, code, cent, _ = o.encode_keys(K, s)
+    lut_sc, _ = o.scores(q, mu, cent, code, s)
+    dense = o.dense_scores(q, K, s)
+    assert np.all(np.isneginf(dense[:s]))
+    assert np.allclose(dense[s:], lut_sc[s:], rtol=1e-12, atol=1e-12)
+    assert np.allclose(dense[s:], K[s:] @ q.sum(axis=0), rtol=0, atol=1e-12)
+
+
+def check_dense_attention(o):
+    import torch
+
+    rng = np.random.default_rng(23)
+    K = rng.standard_normal((300, 16))
+    V = rng.standard_normal((300, 16))
+    q = rng.standard_normal((4, 16))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], torch.from_numpy(K)[None, None].expand(1, 4, -1, -1),
+        torch.from_numpy(V)[None, None].expand(1, 4, -1, -1))[0, :, 0].numpy()
+    assert np.allclose(o.dense_attention(q, K, V), ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(o.dense_attention(q, K, V, 1)[0], V[0], rtol=0, atol=1e-12)       # one token
+    assert np.allclose(o.dense_attention(np.zeros((2, 16)), K, V, 57), V[:57].mean(axis=0)[None].repeat(2, 0),
+                       rtol=0, atol=1e-12)                                               # zero query: mean
+    assert np.all(o.dense_attention(q, K, V, 0) == 0)
+
+
 ALL_CHECKS = [
     check_exact_sum, check_round_to_f32, check_channel_mean, check_sign_codes_golden,
     check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
     check_one_member_clusters_reconstruct, check_scores_golden, check_lut_identity,
     check_topk, check_attention_golden, check_attention_full_selection_is_dense,
     check_attention_invariants, check_needle_recall, check_append_by_construction, check_append_golden,
+    check_dense_scores_equal_lut_scores_when_exact, check_dense_attention,
 ]
