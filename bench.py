@@ -436,6 +436,53 @@ def run_sikv(args):
     del g
     ws.check()
 
+    # comparison baselines on the same workload and replicas (not the method):
+    # full-precision scoring of every token and dense attention over every token
+    n_cmp = min(args.steps, 32)
+    dout = torch.empty_like(out)
+    ws_dscore = sk.Workspace(256, dev, stream)
+    ws_dattn = sk.Workspace(sk.workspace_size("dense_attn", p), dev, stream)
+
+    def dense_score_only(i):
+        c = reps[i % R]
+        sk.sikv_dense_score(p, qs[i], c.K, seq, scores, workspace=ws_dscore, stream=stream)
+
+    def dense_attn_only(i):
+        c = reps[i % R]
+        sk.sikv_dense_attn(p, qs[i], c.K, c.V, seq, dout, workspace=ws_dattn, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            dense_score_only(i)
+            dense_attn_only(i)
+    g = graph_of(dense_score_only, args.warmup, args.warmup + n_cmp)
+    us_dscore = 1e3 * max_over_ranks(timed(g), world) / n_cmp
+    del g
+    g = graph_of(dense_attn_only, args.warmup, args.warmup + n_cmp)
+    us_dattn = 1e3 * max_over_ranks(timed(g), world) / n_cmp
+    del g
+    ws_dscore.check()
+    ws_dattn.check()
+    kv_bytes = K.numel() * K.element_size()
+    comparison = {
+        "note": "own dense kernels on the same GPU and replicas; not the method",
+        "dense_score_us": us_dscore, "lut_score_us": 1e3 * ms_score / args.steps,
+        "retrieval_speedup_lut_vs_dense": us_dscore / (1e3 * ms_score / args.steps),
+        "dense_attention_us": us_dattn, "sikv_decode_us": 1e3 * ms / args.steps,
+        "decode_speedup_sikv_vs_dense_attention": us_dattn / (1e3 * ms / args.steps),
+        "dense_attention_GB_per_s": 2 * kv_bytes / (us_dattn / 1e6) / 1e9,
+        "dense_score_GB_per_s": kv_bytes / (us_dscore / 1e6) / 1e9,
+        # the same ratios against the dense kernels' HBM bound (all of K, or of
+        # K and V, read once at the measured copy peak): independent of how
+        # good the dense kernels are
+        "dense_attention_roofline_us": 2 * kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3),
+        "decode_speedup_sikv_vs_dense_attention_roofline":
+            2 * kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3) / (1e3 * ms / args.steps),
+        "dense_score_roofline_us": kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3),
+        "retrieval_speedup_lut_vs_dense_score_roofline":
+            kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3) / (1e3 * ms_score / args.steps),
+    }
+
     # end to end through the public API: every step is one sikv_decode_host
     # call (a prepared DecodeHostPlan per cache replica) on that step's query
     # and output in page-locked host memory, which the kernels read and write
@@ -506,6 +553,7 @@ def run_sikv(args):
                                   "topk": 1e3 * ms_topk / args.steps, "sparse_attn": 1e3 * ms_attn / args.steps},
         "encode": {"ms": enc_ms, "keys_per_s": w.batch * w.num_kv_heads * w.max_seq_len / (enc_ms / 1e3),
                    "GB_per_s_2reads": 2 * K.numel() * K.element_size() / (enc_ms / 1e3) / 1e9},
+        "comparison": comparison,
         "clocks": sampler.summary(),
         "gpu_launches": launches * args.steps,
         "e2e": e2e,

@@ -127,6 +127,7 @@ SIKV_API size_t sikv_sparse_attn_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_host_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_append_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_dense_attn_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
  * (0 on bad params). */
@@ -245,6 +246,27 @@ SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, 
                                       const uint8_t *codes, const float *codebook, const float *mu,
                                       const int32_t *seq_lens, const int32_t *k_per_seq, void *out_host,
                                       void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+
+/*
+ * Comparison baselines -- not the method.  The pages compare the compressed-
+ * domain retrieval with full dot-product scoring [SIKV 2.1.2] and the sparse
+ * attention with dense attention [SIKV 2.1.4]; these are the library's own
+ * dense kernels for that comparison on the same GPU.  Layouts and errors as
+ * above.
+ *
+ * sikv_dense_score: scores[b][h][t] = q_bar . K[b][h][t] (q_bar the sum of the
+ * group's query heads, fp32 accumulation) for t in [S, N_b), -inf for sinks;
+ * entries t >= N_b are not written.  workspace: the status header (256 B).
+ *
+ * sikv_dense_attn: out[b][hq] = softmax over every token t < N_b of
+ * scale * q . K[t], applied to V, fp32 accumulation, written in the dtype.
+ * workspace: sikv_dense_attn_workspace_size() bytes (split partials).
+ */
+SIKV_API sikv_status sikv_dense_score(const sikv_params *p, const void *q, const void *K, const int32_t *seq_lens,
+                                      float *scores, void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+SIKV_API sikv_status sikv_dense_attn(const sikv_params *p, const void *q, const void *K, const void *V,
+                                     const int32_t *seq_lens, void *out, void *workspace, size_t workspace_bytes,
+                                     sikv_stream_t stream);
 
 /*
  * sikv_sparse_attn_static -- sikv_sparse_attn for callers that cannot

@@ -35,7 +35,8 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
             "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
-            "sikv_append_workspace_size", "sikv_append_codes")
+            "sikv_append_workspace_size", "sikv_append_codes", "sikv_dense_attn_workspace_size",
+            "sikv_dense_score", "sikv_dense_attn")
 
 
 class SikvError(RuntimeError):
@@ -98,7 +99,8 @@ def lib() -> ctypes.CDLL:
         L.sikv_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(i32)]
         for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
                   "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size",
-                  "sikv_decode_host_workspace_size", "sikv_append_workspace_size"):
+                  "sikv_decode_host_workspace_size", "sikv_append_workspace_size",
+                  "sikv_dense_attn_workspace_size"):
             getattr(L, n).restype = sz
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
@@ -110,8 +112,11 @@ def lib() -> ctypes.CDLL:
         L.sikv_decode.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_append_codes.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_dense_score.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_dense_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
-                  "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes"):
+                  "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes",
+                  "sikv_dense_score", "sikv_dense_attn"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -363,3 +368,30 @@ class DecodeHostPlan:
                       self.workspace.nbytes, self._stream)
         if st != 0:
             raise SikvError(st, "sikv_decode_host")
+
+
+# ----------------------------------------------------------------------------
+# comparison baselines (not the method)
+# ----------------------------------------------------------------------------
+
+def sikv_dense_score(p: Params, q, K, seq_lens, scores, workspace=None, stream=None):
+    """Full-precision q_bar . K[t] for every non-sink token (-inf for sinks)."""
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev), _ptr(scores, "scores", torch.float32, (B, H, N), dev))
+    ws = workspace if workspace is not None else Workspace(256, dev, stream)
+    _check(lib().sikv_dense_score(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_dense_score")
+    return ws
+
+
+def sikv_dense_attn(p: Params, q, K, V, seq_lens, out, workspace=None, stream=None):
+    """Dense decode attention over every token of each sequence."""
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(out, "out", p.torch_dtype, (B, p.num_q_heads, D), dev))
+    ws = _ws("dense_attn", p, workspace, dev, stream)
+    _check(lib().sikv_dense_attn(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_dense_attn")
+    return ws

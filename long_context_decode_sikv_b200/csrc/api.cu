@@ -206,6 +206,39 @@ size_t sikv_decode_workspace_size(const sikv_params *p) {
     return decode_layout(*p).total;
 }
 
+size_t sikv_dense_attn_workspace_size(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return sikv::dense_attn_layout(*p, kHeaderBytes).total;
+}
+
+sikv_status sikv_dense_score(const sikv_params *p, const void *q, const void *K, const int32_t *seq_lens,
+                             float *scores, void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(q);
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR4(scores);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, kHeaderBytes));
+    return sikv::launch_dense_score(*p, q, K, seq_lens, scores, reinterpret_cast<int32_t *>(workspace),
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+sikv_status sikv_dense_attn(const sikv_params *p, const void *q, const void *K, const void *V,
+                            const int32_t *seq_lens, void *out, void *workspace, size_t workspace_bytes,
+                            sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(q);
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR(V);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR(out);
+    const sikv::DenseAttnLayout L = sikv::dense_attn_layout(*p, kHeaderBytes);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
+    char *ws = static_cast<char *>(workspace);
+    return sikv::launch_dense_attn(*p, q, K, V, seq_lens, out, ws, kHeaderBytes, reinterpret_cast<int32_t *>(ws),
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t sikv_append_workspace_size(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
     return kHeaderBytes;

@@ -50,6 +50,18 @@ sikv_status launch_encode(const sikv_params &p, const void *K, const int32_t *se
                           uint8_t *codes, float *codebook, int32_t *counts, char *ws,
                           cudaStream_t stream);
 
+// Dense comparison baselines (dense.cu).
+struct DenseAttnLayout {
+    int chunk = 0, nchunks = 0;
+    size_t part_o = 0, part_ml = 0, total = 0;
+};
+DenseAttnLayout dense_attn_layout(const sikv_params &p, size_t base);
+sikv_status launch_dense_score(const sikv_params &p, const void *q, const void *K, const int32_t *seq_lens,
+                               float *scores, int32_t *status, cudaStream_t stream);
+sikv_status launch_dense_attn(const sikv_params &p, const void *q, const void *K, const void *V,
+                              const int32_t *seq_lens, void *out, char *ws, size_t base, int32_t *status,
+                              cudaStream_t stream);
+
 sikv_status launch_append(const sikv_params &p, const void *K, const int32_t *start, const int32_t *count,
                           const float *mu, uint8_t *codes, int32_t *status, cudaStream_t stream);
 sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,
