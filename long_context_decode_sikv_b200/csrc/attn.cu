@@ -62,15 +62,26 @@ attn_partial_kernel(const void *__restrict__ q, const void *__restrict__ K, cons
     for (int e = tid; e < G * kHeadDim; e += kAttnThreads)
         sh.qs[e / kHeadDim][e % kHeadDim] = load1<DT>(qrow, e);
     __syncthreads();
+    // each codebook row is loaded once (all loads of a thread in flight
+    // together) and serves every head of the group
     const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
-    for (int e = tid; e < G * kSubspaces * kClusters; e += kAttnThreads) {
-        const int g = e / (kSubspaces * kClusters), r = e % (kSubspaces * kClusters), s = r >> 4;
-        const float4 c4 = __ldg(cb + r);
-        float v = sh.qs[g][4 * s] * c4.x;
-        v = fmaf(sh.qs[g][4 * s + 1], c4.y, v);
-        v = fmaf(sh.qs[g][4 * s + 2], c4.z, v);
-        v = fmaf(sh.qs[g][4 * s + 3], c4.w, v);
-        sh.lut[g][r] = v;
+    {
+        constexpr int kRows = kSubspaces * kClusters / kAttnThreads;   // 4
+        float4 c4[kRows];
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) c4[i] = __ldg(cb + tid + i * kAttnThreads);
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+            const int r = tid + i * kAttnThreads, s = r >> 4;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float v = sh.qs[g][4 * s] * c4[i].x;
+                v = fmaf(sh.qs[g][4 * s + 1], c4[i].y, v);
+                v = fmaf(sh.qs[g][4 * s + 2], c4[i].z, v);
+                v = fmaf(sh.qs[g][4 * s + 3], c4[i].w, v);
+                sh.lut[g][r] = v;
+            }
+        }
     }
     const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mu + static_cast<size_t>(seg) * kHeadDim) + lane);
     for (int g = warp; g < G; g += kAttnWarps) {
@@ -165,18 +176,31 @@ attn_partial_kernel(const void *__restrict__ q, const void *__restrict__ K, cons
     float o[G][4];
 #pragma unroll
     for (int g = 0; g < G; ++g) o[g][0] = o[g][1] = o[g][2] = o[g][3] = 0.f;
+    // 8 value rows in flight per warp
+    constexpr int kVRows = 8;
     const int n_here = min(kSplit, n_list - p0);
-    for (int i = warp; i < n_here; i += kAttnWarps) {
-        const int t = sh.tok[i];
-        if (t < 0) continue;
-        const float4 v = load4<DT>(static_cast<const char *>(V) + (kv_seg + t) * kHeadDim * EB, lane * 4);
+#pragma unroll 1
+    for (int i0 = warp; i0 < n_here; i0 += kAttnWarps * kVRows) {
+        float4 v[kVRows];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float pv = sh.logit[g][i];
-            o[g][0] = fmaf(pv, v.x, o[g][0]);
-            o[g][1] = fmaf(pv, v.y, o[g][1]);
-            o[g][2] = fmaf(pv, v.z, o[g][2]);
-            o[g][3] = fmaf(pv, v.w, o[g][3]);
+        for (int u = 0; u < kVRows; ++u) {
+            const int i = i0 + u * kAttnWarps;
+            const int t = (i < n_here) ? sh.tok[i] : -1;
+            v[u] = (t >= 0) ? load4<DT>(static_cast<const char *>(V) + (kv_seg + t) * kHeadDim * EB, lane * 4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kVRows; ++u) {
+            const int i = i0 + u * kAttnWarps;
+            if (i >= n_here) break;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float pv = sh.logit[g][i];     // 0 for a skipped entry
+                o[g][0] = fmaf(pv, v[u].x, o[g][0]);
+                o[g][1] = fmaf(pv, v[u].y, o[g][1]);
+                o[g][2] = fmaf(pv, v[u].z, o[g][2]);
+                o[g][3] = fmaf(pv, v[u].w, o[g][3]);
+            }
         }
     }
 #pragma unroll

@@ -13,8 +13,10 @@
 //      radix select on their order-preserving keys finds the exact k-th key T
 //      and how many tokens equal to T are needed (falls back to radix passes
 //      over global memory when bin b* does not fit);
-//   4. one pass in token order emits every key > T and the lowest-index keys
-//      == T, in ascending token order (block prefix sums, no atomics).
+//   4. every key > T and the lowest-index keys == T are emitted in ascending
+//      token order: each warp owns a contiguous run of 32-token groups
+//      (coalesced reads, ballot counts), one scan over the warps places the
+//      runs (no atomics).
 #include "sikv_common.cuh"
 #include "sikv_internal.h"
 
@@ -217,22 +219,59 @@ topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_le
         }
         const uint32_t T = prefix, ties_needed = need;
 
-        // 4. emission in ascending token order
-        uint32_t emitted = 0, ties_seen = 0;
-        for (int base = num_sinks; base < n_tok && emitted < static_cast<uint32_t>(k); base += kTopkThreads) {
-            const int t = base + tid;
-            uint32_t key = 0;
-            const bool valid = t < n_tok;
-            if (valid) key = score_key(srow[t]);
-            const bool eq = valid && key == T;
-            uint32_t eq_tot;
-            const uint32_t eq_rank = ties_seen + block_excl_scan(eq ? 1u : 0u, sh.wtot, &eq_tot);
-            const bool sel = valid && (key > T || (eq && eq_rank < ties_needed));
-            uint32_t sel_tot;
-            const uint32_t pos = emitted + block_excl_scan(sel ? 1u : 0u, sh.wtot, &sel_tot);
-            if (sel && pos < static_cast<uint32_t>(k)) out[pos] = t;
-            emitted += sel_tot;
-            ties_seen += eq_tot;
+        // 4. emission in ascending token order.  Warp w owns a contiguous run
+        // of whole 32-token groups, read with coalesced loads; ballots count
+        // its keys above T and equal to T, one block scan over the warps'
+        // counts places the run, and a second pass over the run writes the
+        // selections in order (a tie is selected while its rank among the
+        // ties, in token order, is below ties_needed).
+        const int groups = (n + 31) / 32;
+        const int gpw = (groups + kTopkWarps - 1) / kTopkWarps;
+        const int t_lo = num_sinks + 32 * min(warp * gpw, groups), t_hi = min(num_sinks + 32 * min((warp + 1) * gpw, groups), n_tok);
+        const uint32_t below = (1u << lane) - 1u;
+        uint32_t c_gt = 0, c_eq = 0;
+#pragma unroll 4
+        for (int t0 = t_lo; t0 < t_hi; t0 += 32) {
+            const int t = t0 + lane;
+            const uint32_t key = t < t_hi ? score_key(srow[t]) : 0u;
+            c_gt += __popc(__ballot_sync(0xffffffffu, t < t_hi && key > T));
+            c_eq += __popc(__ballot_sync(0xffffffffu, t < t_hi && key == T));
+        }
+        // exclusive prefix over the warps of (c_gt, c_eq), packed into one
+        // 64-bit scan done by warp 0
+        if (lane == 0) {
+            sh.hist[2 * warp] = c_gt;
+            sh.hist[2 * warp + 1] = c_eq;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t g = sh.hist[2 * lane], e = sh.hist[2 * lane + 1];
+            uint32_t gi = g, ei = e;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t og = __shfl_up_sync(0xffffffffu, gi, off), oe = __shfl_up_sync(0xffffffffu, ei, off);
+                if (lane >= off) {
+                    gi += og;
+                    ei += oe;
+                }
+            }
+            sh.hist[2 * lane] = gi - g;
+            sh.hist[2 * lane + 1] = ei - e;
+        }
+        __syncthreads();
+        uint32_t tie_rank = sh.hist[2 * warp + 1];
+        uint32_t pos = sh.hist[2 * warp] + min(tie_rank, ties_needed);
+#pragma unroll 1
+        for (int t0 = t_lo; t0 < t_hi; t0 += 32) {
+            const int t = t0 + lane;
+            const uint32_t key = t < t_hi ? score_key(srow[t]) : 0u;
+            const bool gt = t < t_hi && key > T, eq = t < t_hi && key == T;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool tie_sel = eq && tie_rank + __popc(eqm & below) < ties_needed;
+            const uint32_t selm = __ballot_sync(0xffffffffu, gt || tie_sel);
+            if ((gt || tie_sel) && pos + __popc(selm & below) < static_cast<uint32_t>(k)) out[pos + __popc(selm & below)] = t;
+            pos += __popc(selm);
+            tie_rank += __popc(eqm);
         }
     }
     for (int i = k + tid; i < kmax; i += kTopkThreads) out[i] = -1;
