@@ -136,6 +136,29 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
     if (plan.ok)
         return launch_decode_fused(*p, plan, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
                                    scores_out, ws, L.fused, status, s);
+    // Too many segments for one co-resident launch: run the single-launch
+    // kernel on sub-batches of sequences that fit, one after the other on the
+    // stream (each launch leaves the coordination state zeroed for the next).
+    const int bsub = fused_sub_batch(*p);
+    if (bsub > 0) {
+        const size_t eb = p->dtype == SIKV_DTYPE_F32 ? 4 : 2;
+        const size_t hq = p->num_q_heads, hkv = p->num_kv_heads, nmax = p->max_seq_len, d = p->head_dim;
+        for (int b0 = 0; b0 < p->batch; b0 += bsub) {
+            sikv_params ps = *p;
+            ps.batch = std::min(bsub, p->batch - b0);
+            const FusedPlan pl = fused_plan(ps);
+            if (!pl.ok) return SIKV_ERR_UNSUPPORTED;      // cannot happen: fused_sub_batch checked it
+            const size_t bq = static_cast<size_t>(b0) * hq * d * eb, bkv = static_cast<size_t>(b0) * hkv * nmax * d * eb;
+            SIKV_TRY(launch_decode_fused(
+                ps, pl, static_cast<const char *>(q) + bq, static_cast<const char *>(K) + bkv,
+                static_cast<const char *>(V) + bkv, codes + static_cast<size_t>(b0) * hkv * nmax * (d / 8),
+                codebook + static_cast<size_t>(b0) * hkv * kSubspaces * kClusters * 4,
+                mu + static_cast<size_t>(b0) * hkv * d, seq_lens + b0, k_per_seq + b0, static_cast<char *>(out) + bq,
+                idx_out ? idx_out + static_cast<size_t>(b0) * hkv * (p->max_topk > 0 ? p->max_topk : 0) : nullptr,
+                scores_out ? scores_out + static_cast<size_t>(b0) * hkv * nmax : nullptr, ws, L.fused, status, s));
+        }
+        return SIKV_OK;
+    }
     float *sc = scores_out ? scores_out : reinterpret_cast<float *>(ws + L.scores);
     int32_t *ix = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     SIKV_TRY(launch_score(*p, q, codes, codebook, mu, seq_lens, sc, status, s));
@@ -266,6 +289,8 @@ size_t sikv_decode_host_workspace_size(const sikv_params *p) {
 int32_t sikv_decode_launches(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
     if (fused_plan(*p).ok) return 1;               // one cooperative kernel
+    const int bsub = fused_sub_batch(*p);
+    if (bsub > 0) return (p->batch + bsub - 1) / bsub;   // one per sub-batch
     return 1 + (p->max_topk > 0 ? 1 : 0) + 2;     // score, top-k, attention partials + combine
 }
 

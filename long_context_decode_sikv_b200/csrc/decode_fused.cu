@@ -1203,6 +1203,17 @@ FusedPlan fused_plan(const sikv_params &p) {
     return plan;
 }
 
+int fused_sub_batch(const sikv_params &p) {
+    // the largest number of sequences per launch whose segments fit one
+    // co-resident launch (0: none does, or the whole batch already does)
+    for (int bs = p.batch - 1; bs >= 1; --bs) {
+        sikv_params ps = p;
+        ps.batch = bs;
+        if (fused_plan(ps).ok) return bs;
+    }
+    return 0;
+}
+
 sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
                                 const void *V, const uint8_t *codes, const float *codebook, const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,

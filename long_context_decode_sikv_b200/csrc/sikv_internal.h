@@ -97,6 +97,7 @@ struct FusedPlan {
 
 FusedLayout fused_layout(const sikv_params &p, size_t base);
 FusedPlan fused_plan(const sikv_params &p);
+int fused_sub_batch(const sikv_params &p);   // sequences per launch when the batch must be split; 0: no split
 sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
                                 const void *V, const uint8_t *codes, const float *codebook, const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,

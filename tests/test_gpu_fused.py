@@ -138,3 +138,37 @@ def test_decode_host_matches_device_decode(name):
         torch.cuda.synchronize()
         assert plan.workspace.check() == 0
         assert torch.equal(oh2, out_d.cpu()), (name, step)
+
+
+def test_batch_split_into_sub_launches_matches_oracle():
+    """More segments than one co-resident launch holds at this length: the
+    batch runs as consecutive single-launch sub-batches (here 18 + 1
+    sequences), each checked against the oracle on a sampled segment."""
+    dev = gu.device()
+    B, H, N, S, k = 19, 8, 16896, 64, 842
+    p = sk.make_params("bf16", B, H, H, N, S, k)
+    assert int(sk.lib().sikv_decode_launches(ctypes.byref(p))) == 2
+    g = torch.Generator().manual_seed(31)
+    K = torch.randn((B, H, N, 128), generator=g).to(torch.bfloat16)
+    V = torch.randn((B, H, N, 128), generator=g).to(torch.bfloat16)
+    q = torch.randn((B, H, 128), generator=g).to(torch.bfloat16)
+    seq = torch.full((B,), N, dtype=torch.int32, device=dev)
+    kk = torch.full((B,), k, dtype=torch.int32, device=dev)
+    c = sk.SikvCache(p, K.to(dev), V.to(dev), seq)
+    c.encode()
+    out = torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)
+    idx = torch.full((B, H, k), -7, dtype=torch.int32, device=dev)
+    c.decode(q.to(dev), kk, out=out, idx_out=idx)
+    torch.cuda.synchronize()
+    c.check()
+    idx = idx.cpu().numpy()
+    out = gu.to_f64(out)
+    for b, h in ((0, 0), (17, 5), (18, 7)):
+        Kb = K[b, h].double().numpy()
+        Vb = V[b, h].double().numpy()
+        qb = q[b, h:h + 1].double().numpy()
+        mu, code, cent, _ = oracle.encode_keys(Kb, S)
+        o_out, o_idx, o_sc, cond = oracle.decode_step(qb, Kb, Vb, mu, cent, code, k, S)
+        assert np.all(np.diff(idx[b, h]) > 0)
+        gu.check_selection(idx[b, h], o_idx, o_sc, cond, k)
+        assert np.allclose(out[b, h:h + 1], o_out, atol=2e-2, rtol=1e-2), (b, h)
