@@ -250,7 +250,8 @@ SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, 
 /*
  * Comparison baselines -- not the method.  The pages compare the compressed-
  * domain retrieval with full dot-product scoring [SIKV 2.1.2] and the sparse
- * attention with dense attention [SIKV 2.1.4]; these are the library's own
+ * attention with dense attention [SIKV 2.1.4], and quote the speed-ups of
+ * both in their efficiency results [SIKV 4]; these are the library's own
  * dense kernels for that comparison on the same GPU.  Layouts and errors as
  * above.
  *
