@@ -47,6 +47,25 @@ R14 a selected key is reconstructed as mu + c[s][code_s];
 R19 a token appended at decode time is coded against the prefill mean, which
     stays frozen;
 R20 the codebook stays frozen too: appended tokens do not move the centroids.
+
+The k-means codebook (a comparison baseline, not the method: the iterative
+clustering that [SIKV §2.1.1]'s one-pass clustering replaces, timed against it
+with 20 iterations in [SIKV §4]) adds:
+
+R21 k-means clusters the same points as the one-pass codebook: the normalized
+    sub-vectors x = fl32(k - mu) of the non-sink tokens, 16 clusters per
+    subspace, Lloyd's iterations (assign every point to its nearest centroid,
+    then move every centroid to the mean of its points);
+R22 initialization picks 16 distinct non-sink tokens (drawn by the seeded
+    input generator and passed in); centroid j of subspace s starts at token
+    j's sub-vector s;
+R23 the nearest centroid minimizes the squared distance
+    ((d0*d0 + d1*d1) + d2*d2) + d3*d3 with d_i = x_i - c_i, every operation
+    rounded to fp32 in that order (no fused multiply-add); ties go to the
+    lower cluster index;
+R24 a non-empty cluster's new centroid is the exact mean of its points,
+    rounded once to fp32; an empty cluster keeps its centroid.  After the last
+    iteration the codes are its assignment and the counts its cluster sizes.
 """
 
 from __future__ import annotations
@@ -59,6 +78,7 @@ import numpy as np
 SUB_DIM = 4          # [SIKV §2.1.1]: 4-dimensional sub-vectors
 NUM_CLUSTERS = 16    # [SIKV §2.1.1]: sign pattern of 4 dims -> one of 16 clusters
 DEFAULT_SINKS = 64   # [SIKV §2.1.3]: 64 full-precision sink tokens
+KMEANS_ITERS = 20    # [SIKV §4]: the k-means the one-pass clustering is timed against
 
 
 # ----------------------------------------------------------------------------
@@ -333,6 +353,82 @@ def dense_attention(q_group: np.ndarray, K: np.ndarray, V: np.ndarray, n_tok: in
     p = np.exp(logits - m)
     p /= p.sum(axis=1, keepdims=True)
     return p @ V[:n]
+
+
+# ----------------------------------------------------------------------------
+# comparison baseline: k-means codebook  [SIKV §2.1.1, §4]  (R21-R24)
+# ----------------------------------------------------------------------------
+
+def kmeans_points(K: np.ndarray, mu: np.ndarray, num_sinks: int = DEFAULT_SINKS) -> np.ndarray:
+    """The points k-means clusters (R21): x[t, s] = fl32(K[t, 4s:4s+4] - mu[4s:4s+4])
+    for the non-sink tokens, float32 [N - S][P][4].  Stored keys are exact in fp32.
+    """
+    K32 = np.asarray(K, dtype=np.float64).astype(np.float32)
+    mu32 = np.asarray(mu, dtype=np.float32)
+    n_tok, d = K32.shape
+    x = K32[num_sinks:] - mu32[None, :]                 # one fp32 subtraction each
+    return x.reshape(max(n_tok - num_sinks, 0), d // SUB_DIM, SUB_DIM)
+
+
+def kmeans_assign(x: np.ndarray, cent: np.ndarray) -> np.ndarray:
+    """Nearest centroid of every point (R23).  x float32 [n][P][4], cent float32
+    [P][16][4]; returns uint8 [n][P].  numpy rounds each float32 operation on its
+    own, and argmin returns the first of equal minima (the lower index).
+    """
+    out = np.zeros(x.shape[:2], dtype=np.uint8)
+    for t0 in range(0, x.shape[0], 4096):
+        diff = x[t0:t0 + 4096, :, None, :] - cent[None, :, :, :]          # [n][P][16][4]
+        sq = diff * diff
+        dist = ((sq[..., 0] + sq[..., 1]) + sq[..., 2]) + sq[..., 3]
+        out[t0:t0 + 4096] = np.argmin(dist, axis=2)
+    return out
+
+
+def kmeans_update(x: np.ndarray, assign: np.ndarray, cent: np.ndarray):
+    """Move every non-empty centroid to the exact mean of its points, rounded
+    once to fp32; empty clusters keep theirs (R24).  Returns (centroids float32
+    [P][16][4], counts int64 [P][16]).
+    """
+    p = x.shape[1]
+    new = np.array(cent, dtype=np.float32, copy=True)
+    counts = np.zeros((p, NUM_CLUSTERS), dtype=np.int64)
+    for s in range(p):
+        for j in range(NUM_CLUSTERS):
+            members = x[assign[:, s] == j, s, :]
+            counts[s, j] = members.shape[0]
+            if members.shape[0]:
+                for i in range(SUB_DIM):
+                    new[s, j, i] = round_to_f32(exact_sum(members[:, i].tolist()) / members.shape[0])
+    return new, counts
+
+
+def kmeans_codebook(K: np.ndarray, mu: np.ndarray, init_idx, iters: int = KMEANS_ITERS,
+                    num_sinks: int = DEFAULT_SINKS):
+    """K-means codebook of one (sequence, KV head), the iterative baseline of
+    [SIKV §2.1.1] (R21-R24): ``iters`` Lloyd's iterations from the centroids at
+    the 16 tokens ``init_idx``.
+
+    Returns (codes uint8 [N][P] one nibble per entry, rows t < S zero;
+    centroids float32 [P][16][4]; counts int64 [P][16]).  With no non-sink
+    token every centroid and count is 0.
+    """
+    if iters < 1:
+        raise ValueError("k-means needs at least one iteration")
+    n_tok, d = np.asarray(K).shape
+    p = d // SUB_DIM
+    code = np.zeros((n_tok, p), dtype=np.uint8)
+    x = kmeans_points(K, mu, num_sinks)
+    if x.shape[0] == 0:
+        return code, np.zeros((p, NUM_CLUSTERS, SUB_DIM), dtype=np.float32), np.zeros((p, NUM_CLUSTERS), np.int64)
+    idx = np.asarray(init_idx, dtype=np.int64)
+    if idx.shape != (NUM_CLUSTERS,) or np.any(idx < num_sinks) or np.any(idx >= n_tok):
+        raise ValueError("init_idx must hold 16 non-sink token positions")
+    cent = np.ascontiguousarray(x[idx - num_sinks].transpose(1, 0, 2))   # [P][16][4]
+    for _ in range(iters):
+        assign = kmeans_assign(x, cent)
+        cent, counts = kmeans_update(x, assign, cent)
+    code[num_sinks:] = assign
+    return code, cent, counts
 
 
 def decode_step(q_group, K, V, mu, centroids, code, k, num_sinks=DEFAULT_SINKS, scale=None):

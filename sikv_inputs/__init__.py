@@ -49,6 +49,7 @@ ROLE_NEEDLES = 4
 ROLE_LENGTHS = 5
 ROLE_SCORES = 6
 ROLE_INDICES = 7
+ROLE_KMEANS_INIT = 8
 
 
 # ----------------------------------------------------------------------------
@@ -333,3 +334,17 @@ def random_indices(seed: int, seq_len: int, num_sinks: int, k: int) -> np.ndarra
     """k distinct token positions in [num_sinks, seq_len), in random order."""
     rng = np.random.default_rng(np.random.SeedSequence([seed, seq_len, k, ROLE_INDICES, 0]))
     return (rng.choice(seq_len - num_sinks, size=k, replace=False) + num_sinks).astype(np.int32)
+
+
+def kmeans_init(w: Workload, seq_lens, clusters: int = 16) -> np.ndarray:
+    """Starting tokens of the k-means baseline: for every (sequence b, KV head
+    h), ``clusters`` distinct positions drawn uniformly from [num_sinks,
+    seq_lens[b]), in random order; int32 [B][Hkv][clusters]."""
+    out = np.zeros((w.batch, w.num_kv_heads, clusters), dtype=np.int32)
+    for b in range(w.batch):
+        n = int(seq_lens[b]) - w.num_sinks
+        if n < clusters:
+            raise ValueError(f"sequence {b} has {n} non-sink tokens, fewer than {clusters}")
+        for h in range(w.num_kv_heads):
+            out[b, h] = _rng(w, b, h, ROLE_KMEANS_INIT).choice(n, size=clusters, replace=False) + w.num_sinks
+    return out

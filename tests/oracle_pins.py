@@ -435,6 +435,99 @@ def check_dense_attention(o):
     assert np.all(o.dense_attention(q, K, V, 0) == 0)
 
 
+
+
+# --------------------------------------------------------------------------
+# k-means codebook baseline (§2.1 item 1: the iterative clustering that the
+# one-pass sign-pattern clustering replaces; §4: timed with 20 iterations)
+# --------------------------------------------------------------------------
+
+def _corner(j):
+    return [1.0 if (j >> i) & 1 else -1.0 for i in range(4)]
+
+
+def check_kmeans_golden(o):
+    g = _load("kmeans_d8.json")
+    s = g["num_sinks"]
+    mu = np.array(g["mu"], dtype=np.float32)
+    x = np.array(g["x"], dtype=np.float64).reshape(len(g["x"]), 8)
+    K = x + mu.astype(np.float64)[None, :]
+    want_cent = np.array([[_corner(j) for j in range(16)] for _ in range(2)], dtype=np.float32)
+    for sub, cs in g["centroids_not_on_corner"].items():
+        for j, c in cs.items():
+            want_cent[int(sub), int(j)] = c
+    for iters in g["iters"]:
+        code, cent, counts = o.kmeans_codebook(K, mu, g["init_idx"], iters, s)
+        assert np.array_equal(code, np.array(g["codes"], dtype=np.uint8)), iters
+        assert np.array_equal(counts, np.array(g["counts"])), iters
+        assert cent.dtype == np.float32 and np.array_equal(cent, want_cent), iters
+
+
+def check_kmeans_update_exact(o):
+    """A centroid is the exact mean rounded once: 2**30 + 2**-30 - 2**30 loses
+    its middle term in any fp64 running sum."""
+    x = np.zeros((3, 1, 4), dtype=np.float32)
+    x[:, 0, 0] = [2.0 ** 30, 2.0 ** -30, -(2.0 ** 30)]
+    x[:, 0, 1] = [1.0, 2.0, 4.0]
+    x[:, 0, 2] = [0.1, 0.2, 0.3]
+    cent0 = np.arange(64, dtype=np.float32).reshape(1, 16, 4)
+    cent, counts = o.kmeans_update(x, np.zeros((3, 1), dtype=np.uint8), cent0)
+    assert counts.tolist() == [[3] + [0] * 15]
+    assert cent[0, 0, 0] == np.float32(float(Fraction(1, 3 * 2 ** 30)))
+    assert cent[0, 0, 1] == np.float32(7.0 / 3.0)
+    exact = sum(Fraction(float(v)) for v in x[:, 0, 2]) / 3
+    assert abs(Fraction(float(cent[0, 0, 2])) - exact) <= Fraction(float(np.spacing(np.float32(0.2)))) / 2
+    assert cent[0, 0, 3] == 0.0
+    assert np.array_equal(cent[0, 1:], cent0[0, 1:])               # empty clusters keep theirs
+
+
+def _kmeans_data(seed=31, n=400, s=3):
+    rng = np.random.default_rng(seed)
+    K = (rng.standard_normal((n + s, 8)) * 1.5 + rng.standard_normal(8)).astype(np.float32).astype(np.float64)
+    mu = rng.standard_normal(8).astype(np.float32)
+    init = rng.choice(np.arange(s, n + s), size=16, replace=False)
+    return K, mu, init, s
+
+
+def check_kmeans_matches_sklearn(o):
+    """Lloyd's iterations from the same start agree with scikit-learn's
+    KMeans (lloyd, fp64, no early stop) on points with no empty cluster."""
+    from sklearn.cluster import KMeans
+
+    K, mu, init, s = _kmeans_data()
+    x = (K.astype(np.float32)[s:] - mu[None, :]).astype(np.float64)
+    for iters in (1, 3):
+        code, cent, counts = o.kmeans_codebook(K, mu, init, iters, s)
+        assert np.all(counts > 0)
+        for sub in range(2):
+            pts = x[:, 4 * sub:4 * sub + 4]
+            km = KMeans(n_clusters=16, init=pts[init - s], n_init=1, max_iter=iters, tol=0.0,
+                        algorithm="lloyd").fit(pts)
+            assert np.allclose(cent[sub], km.cluster_centers_, rtol=0, atol=1e-5), (iters, sub)
+
+
+def check_kmeans_lloyd_invariants(o):
+    """Cluster sizes add up to n, every centroid is the mean of its points, the
+    codes of sinks are 0, and the within-cluster sum of squares never grows
+    from one iteration to the next."""
+    K, mu, init, s = _kmeans_data(seed=37)
+    x = (K.astype(np.float32)[s:] - mu[None, :]).astype(np.float64)
+    prev = None
+    for iters in range(1, 7):
+        code, cent, counts = o.kmeans_codebook(K, mu, init, iters, s)
+        assert np.all(code[:s] == 0) and np.all(counts.sum(axis=1) == x.shape[0])
+        sse = 0.0
+        for sub in range(2):
+            pts = x[:, 4 * sub:4 * sub + 4]
+            lab = code[s:, sub]
+            assert np.array_equal(np.bincount(lab, minlength=16), counts[sub])
+            for j in range(16):
+                if counts[sub, j]:
+                    assert np.allclose(cent[sub, j], pts[lab == j].mean(axis=0), rtol=1e-6, atol=1e-6)
+            sse += float(((pts - cent[sub][lab].astype(np.float64)) ** 2).sum())
+        assert prev is None or sse <= prev * (1 + 1e-6), (iters, sse, prev)
+        prev = sse
+
 ALL_CHECKS = [
     check_exact_sum, check_round_to_f32, check_channel_mean, check_sign_codes_golden,
     check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
@@ -442,4 +535,6 @@ ALL_CHECKS = [
     check_topk, check_attention_golden, check_attention_full_selection_is_dense,
     check_attention_invariants, check_needle_recall, check_append_by_construction, check_append_golden,
     check_dense_scores_equal_lut_scores_when_exact, check_dense_attention,
+    check_kmeans_golden, check_kmeans_update_exact, check_kmeans_matches_sklearn,
+    check_kmeans_lloyd_invariants,
 ]

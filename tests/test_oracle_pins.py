@@ -90,6 +90,50 @@ def _mut_append_one_row_too_many(packed, K, mu, start, count):
         else oracle.append_codes(packed, K, mu, start, count)
 
 
+def _mut_kmeans_ties_high(x, cent):
+    diff = x[:, :, None, :] - cent[None, :, :, :]
+    sq = diff * diff
+    dist = ((sq[..., 0] + sq[..., 1]) + sq[..., 2]) + sq[..., 3]
+    return (15 - np.argmin(dist[:, :, ::-1], axis=2)).astype(np.uint8)
+
+
+def _mut_kmeans_l1(x, cent):
+    dist = np.abs(x[:, :, None, :] - cent[None, :, :, :]).sum(axis=3)
+    return np.argmin(dist, axis=2).astype(np.uint8)
+
+
+def _mut_kmeans_empty_zero(x, assign, cent):
+    new, counts = oracle.kmeans_update(x, assign, cent)
+    new[counts == 0] = 0.0
+    return new, counts
+
+
+def _mut_kmeans_fp64_mean(x, assign, cent):
+    new = np.array(cent, dtype=np.float32, copy=True)
+    counts = np.zeros((x.shape[1], 16), dtype=np.int64)
+    for s in range(x.shape[1]):
+        for j in range(16):
+            m = x[assign[:, s] == j, s, :].astype(np.float64)
+            counts[s, j] = m.shape[0]
+            if m.shape[0]:
+                new[s, j] = m.mean(axis=0).astype(np.float32)
+    return new, counts
+
+
+def _mut_kmeans_no_mu(K, mu, num_sinks=64):
+    return oracle.kmeans_points(K, np.zeros_like(np.asarray(mu, dtype=np.float32)), num_sinks)
+
+
+def _mut_kmeans_with_sinks(K, mu, init_idx, iters=20, num_sinks=64):
+    code, cent, counts = oracle.kmeans_codebook(K, mu, init_idx, iters, 0)
+    code[:num_sinks] = 0
+    return code, cent, counts
+
+
+def _mut_kmeans_one_short(K, mu, init_idx, iters=20, num_sinks=64):
+    return oracle.kmeans_codebook(K, mu, init_idx, max(iters - 1, 1), num_sinks)
+
+
 MUTATIONS = {
     "strict-greater": dict(sign_codes=_mut_codes_strict),
     "msb-first-bits": dict(sign_codes=_mut_codes_msb_first),
@@ -102,6 +146,13 @@ MUTATIONS = {
     "dropped-q-dot-mu": dict(scores=_mut_scores_no_qmu),
     "append-reestimates-mean": dict(append_codes=_mut_append_reestimates_mean),
     "append-one-row-too-many": dict(append_codes=_mut_append_one_row_too_many),
+    "kmeans-ties-to-higher-index": dict(kmeans_assign=_mut_kmeans_ties_high),
+    "kmeans-l1-distance": dict(kmeans_assign=_mut_kmeans_l1),
+    "kmeans-empty-cluster-to-zero": dict(kmeans_update=_mut_kmeans_empty_zero),
+    "kmeans-plain-fp64-mean": dict(kmeans_update=_mut_kmeans_fp64_mean),
+    "kmeans-no-mean-normalization": dict(kmeans_points=_mut_kmeans_no_mu),
+    "kmeans-clusters-sinks": dict(kmeans_codebook=_mut_kmeans_with_sinks),
+    "kmeans-one-iteration-short": dict(kmeans_codebook=_mut_kmeans_one_short),
 }
 
 
