@@ -483,6 +483,39 @@ def run_sikv(args):
             kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3) / (1e3 * ms_score / args.steps),
     }
 
+    # clustering: the one-pass sign-pattern codebook (the whole prefill
+    # encoder, mean pass included) against 20 Lloyd's k-means iterations on the
+    # same points (mean given), both on this GPU with this library's kernels
+    init = torch.from_numpy(gen.kmeans_init(w, w.seq_lens)).to(dev)
+    km_codes, km_cb, km_cnt = torch.empty_like(base.codes), torch.empty_like(base.codebook), torch.empty_like(base.counts)
+    ws_km = sk.Workspace(sk.workspace_size("kmeans", p), dev, stream)
+
+    def kmeans20():
+        sk.sikv_kmeans_codebook(p, K, seq, base.mu, init, km_codes, km_cb, km_cnt, iters=20, workspace=ws_km,
+                                stream=stream)
+
+    with torch.cuda.stream(stream):
+        kmeans20()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(2):
+            kmeans20()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    km_ms = max_over_ranks(a.elapsed_time(b), world) / 2
+    ws_km.check()
+    comparison.update({
+        "one_pass_encode_ms": enc_ms, "kmeans20_ms": km_ms,
+        "clustering_speedup_one_pass_vs_kmeans20": km_ms / enc_ms,
+        "kmeans_iteration_us": 1e3 * km_ms / 20,
+        "kmeans_iteration_key_GB_per_s": K.numel() * K.element_size() / (km_ms / 20 / 1e3) / 1e9,
+    })
+    del km_codes, km_cb, km_cnt, ws_km
+
     # end to end through the public API: every step is one sikv_decode_host
     # call (a prepared DecodeHostPlan per cache replica) on that step's query
     # and output in page-locked host memory, which the kernels read and write

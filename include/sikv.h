@@ -128,6 +128,7 @@ SIKV_API size_t sikv_decode_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_decode_host_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_append_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_dense_attn_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_kmeans_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
  * (0 on bad params). */
@@ -268,6 +269,42 @@ SIKV_API sikv_status sikv_dense_score(const sikv_params *p, const void *q, const
 SIKV_API sikv_status sikv_dense_attn(const sikv_params *p, const void *q, const void *K, const void *V,
                                      const int32_t *seq_lens, void *out, void *workspace, size_t workspace_bytes,
                                      sikv_stream_t stream);
+
+/*
+ * sikv_kmeans_codebook -- comparison baseline, not the method: the iterative
+ * K-means clustering that the one-pass sign-pattern codebook replaces
+ * [SIKV 2.1.1], timed against it with 20 iterations [SIKV 4].  The pages
+ * give no K-means details; this is Lloyd's algorithm on the same points and
+ * codebook shape, for every (b, h):
+ *   points  x[t][s] = fl32(K[t][4s:4s+4] - mu[4s:4s+4]) for t in [S, N_b);
+ *   start   c[s][j] = x[init_idx[b][h][j]][s] for j < 16;
+ *   iters   times: assign every point to the nearest centroid, minimizing
+ *           ((d0*d0 + d1*d1) + d2*d2) + d3*d3 with d_i = x_i - c_i, each
+ *           operation rounded to fp32 in that order, ties to the lower j;
+ *           then move each non-empty cluster to the exact mean of its points
+ *           rounded once to fp32 (an empty cluster keeps its centroid).
+ * Outputs, in the layouts of sikv_encode_keys so that sikv_score reads them:
+ *  - codes: device u8 [B][Hkv][Nmax][D/8]; rows t in [S, N_b) receive the
+ *    last assignment, two codes per byte, even subspace in the low nibble;
+ *    other rows are not written.
+ *  - codebook: device fp32 [B][Hkv][D/4][16][4], the final centroids; it also
+ *    holds the centroids between iterations.
+ *  - counts: device int32 [B][Hkv][D/4][16], the last cluster sizes (may be NULL).
+ * Inputs: K (dtype) [B][Hkv][Nmax][D], seq_lens [B], mu fp32 [B][Hkv][D] (the
+ * channel mean of sikv_encode_keys), init_idx int32 [B][Hkv][16] (distinct
+ * tokens in [S, N_b), drawn by the caller).  1 <= iters <= 1000, else
+ * SIKV_ERR_INVALID_ARG.  Errors: an invalid seq_lens[b] sets
+ * SIKV_DEVERR_SEQ_LEN and a start token outside [S, N_b) sets
+ * SIKV_DEVERR_INDEX (its centroids start at 0); a sequence with N_b <= S
+ * gets centroids 0 and counts 0.  The sums are exact while a cluster's
+ * points span fewer than about 40 binades.
+ *  - workspace: sikv_kmeans_workspace_size() bytes (chunk partials), on the
+ *    device that runs the call.
+ */
+SIKV_API sikv_status sikv_kmeans_codebook(const sikv_params *p, const void *K, const int32_t *seq_lens,
+                                          const float *mu, const int32_t *init_idx, int32_t iters, uint8_t *codes,
+                                          float *codebook, int32_t *counts, void *workspace, size_t workspace_bytes,
+                                          sikv_stream_t stream);
 
 /*
  * sikv_sparse_attn_static -- sikv_sparse_attn for callers that cannot

@@ -36,7 +36,7 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
             "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
             "sikv_append_workspace_size", "sikv_append_codes", "sikv_dense_attn_workspace_size",
-            "sikv_dense_score", "sikv_dense_attn")
+            "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_workspace_size", "sikv_kmeans_codebook")
 
 
 class SikvError(RuntimeError):
@@ -100,7 +100,7 @@ def lib() -> ctypes.CDLL:
         for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
                   "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size",
                   "sikv_decode_host_workspace_size", "sikv_append_workspace_size",
-                  "sikv_dense_attn_workspace_size"):
+                  "sikv_dense_attn_workspace_size", "sikv_kmeans_workspace_size"):
             getattr(L, n).restype = sz
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
@@ -114,9 +114,10 @@ def lib() -> ctypes.CDLL:
         L.sikv_append_codes.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_dense_score.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_dense_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_kmeans_codebook.argtypes = [pp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
                   "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes",
-                  "sikv_dense_score", "sikv_dense_attn"):
+                  "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_codebook"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -246,6 +247,24 @@ def sikv_append_codes(p: Params, K, start, count, mu, codes, workspace=None, str
     ws = _ws("append", p, workspace, dev, stream)
     _check(lib().sikv_append_codes(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)),
            "sikv_append_codes")
+    return ws
+
+
+def sikv_kmeans_codebook(p: Params, K, seq_lens, mu, init_idx, codes, codebook, counts=None, iters=20,
+                         workspace=None, stream=None):
+    """Comparison baseline: ``iters`` Lloyd's k-means iterations on the
+    normalized sub-vectors from the start tokens ``init_idx`` [B][Hkv][16];
+    codes, centroids and counts in the layouts of :func:`sikv_encode_keys`."""
+    dev = K.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(K, "K", p.torch_dtype, (B, H, N, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(init_idx, "init_idx", torch.int32, (B, H, 16), dev))
+    outs = (_ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(counts, "counts", torch.int32, (B, H, D // 4, 16), dev, optional=True))
+    ws = _ws("kmeans", p, workspace, dev, stream)
+    _check(lib().sikv_kmeans_codebook(ctypes.byref(p), *args, int(iters), *outs, ws.ptr, ws.nbytes,
+                                      _stream(stream, dev)), "sikv_kmeans_codebook")
     return ws
 
 

@@ -281,6 +281,29 @@ sikv_status sikv_append_codes(const sikv_params *p, const void *K, const int32_t
     return sikv::launch_append(*p, K, start, count, mu, codes, status, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t sikv_kmeans_workspace_size(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return sikv::kmeans_layout(*p, device_sm_count()).total;
+}
+
+sikv_status sikv_kmeans_codebook(const sikv_params *p, const void *K, const int32_t *seq_lens, const float *mu,
+                                 const int32_t *init_idx, int32_t iters, uint8_t *codes, float *codebook,
+                                 int32_t *counts, void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR(mu);
+    SIKV_REQUIRE_PTR4(init_idx);
+    SIKV_REQUIRE_PTR(codes);
+    SIKV_REQUIRE_PTR(codebook);
+    if (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)) return SIKV_ERR_UNSUPPORTED;
+    if (iters < 1 || iters > 1000) return SIKV_ERR_INVALID_ARG;
+    const sikv::KmeansLayout L = sikv::kmeans_layout(*p, device_sm_count());
+    SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
+    return sikv::launch_kmeans(*p, L, K, seq_lens, mu, init_idx, iters, codes, codebook, counts,
+                               static_cast<char *>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t sikv_decode_host_workspace_size(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
     return sikv::host_layout(*p, decode_layout(*p).total).total;

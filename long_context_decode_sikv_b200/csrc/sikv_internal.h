@@ -62,6 +62,16 @@ sikv_status launch_dense_attn(const sikv_params &p, const void *q, const void *K
                               const int32_t *seq_lens, void *out, char *ws, size_t base, int32_t *status,
                               cudaStream_t stream);
 
+// K-means codebook baseline (kmeans.cu).
+struct KmeansLayout {
+    int chunk = 0, nchunks = 0;           // tokens per CTA, CTAs per segment
+    size_t part_sum = 0, part_cnt = 0, total = 0;
+};
+KmeansLayout kmeans_layout(const sikv_params &p, int num_sms);
+sikv_status launch_kmeans(const sikv_params &p, const KmeansLayout &L, const void *K, const int32_t *seq_lens,
+                          const float *mu, const int32_t *init_idx, int iters, uint8_t *codes, float *codebook,
+                          int32_t *counts, char *ws, cudaStream_t stream);
+
 sikv_status launch_append(const sikv_params &p, const void *K, const int32_t *start, const int32_t *count,
                           const float *mu, uint8_t *codes, int32_t *status, cudaStream_t stream);
 sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,

@@ -140,3 +140,20 @@ def test_append_validates_without_launch():
     assert L.sikv_append_codes(ctypes.byref(p), fake, None, fake, fake, fake, fake, 256, None) == 1
     assert L.sikv_append_codes(ctypes.byref(p), fake, fake, fake, fake, None, fake, 256, None) == 1
     assert L.sikv_append_codes(ctypes.byref(p), fake, fake, fake, fake, fake, fake, 16, None) == 3   # workspace too small
+
+
+def test_kmeans_validates_without_launch():
+    p = _p()
+    L = sk.lib()
+    assert L.sikv_kmeans_workspace_size(ctypes.byref(p)) > 256
+    fake = ctypes.c_void_p(1 << 20)
+    ws = L.sikv_kmeans_workspace_size(ctypes.byref(p))
+    args = [fake, fake, fake, fake]
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), None, *args[1:], 20, fake, fake, None, fake, ws, None) == 1
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args[:3], None, 20, fake, fake, None, fake, ws, None) == 1
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 20, None, fake, None, fake, ws, None) == 1
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 0, fake, fake, None, fake, ws, None) == 1      # iters < 1
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 1001, fake, fake, None, fake, ws, None) == 1   # iters > 1000
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 20, fake, fake, ctypes.c_void_p((1 << 20) + 2),
+                                  fake, ws, None) == 2                                                  # misaligned counts
+    assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 20, fake, fake, None, fake, 256, None) == 3   # workspace too small
