@@ -66,6 +66,22 @@ R23 the nearest centroid minimizes the squared distance
 R24 a non-empty cluster's new centroid is the exact mean of its points,
     rounded once to fp32; an empty cluster keeps its centroid.  After the last
     iteration the codes are its assignment and the counts its cluster sizes.
+
+The 2-bit value operating point (the pages say accuracy holds with 2-bit
+quantization and that the memory saving matches 2-bit KIVI [SIKV §3, §4], but
+give no scheme) adds:
+
+R25 V is quantized per token in groups of 32 channels, asymmetrically: a group
+    keeps its minimum m and step s = (max - min) / 3, a value its level
+    q in {0, 1, 2, 3}, and reads back as m + q s (KIVI's per-token value
+    quantization);
+R26 m and s are stored in fp16 (round to nearest even) after s is formed in
+    fp32 as fl32(fl32(max - min) / 3); the level is
+    clamp(rint(fl32(fl32(v - m16) / s16)), 0, 3) in fp32 with ties to even,
+    and 0 when s16 = 0; values must lie in the fp16 range;
+R27 sinks keep their full-precision V; only selected tokens read quantized V;
+R28 a token's quantized row is 48 bytes: 32 bytes of levels (dimension d in
+    bits 2 (d mod 4) of byte d / 4), then (m16, s16) of groups 0..3.
 """
 
 from __future__ import annotations
@@ -79,6 +95,8 @@ SUB_DIM = 4          # [SIKV §2.1.1]: 4-dimensional sub-vectors
 NUM_CLUSTERS = 16    # [SIKV §2.1.1]: sign pattern of 4 dims -> one of 16 clusters
 DEFAULT_SINKS = 64   # [SIKV §2.1.3]: 64 full-precision sink tokens
 KMEANS_ITERS = 20    # [SIKV §4]: the k-means the one-pass clustering is timed against
+V_GROUP = 32         # R25: channels per quantization group of a value row
+V_ROW_BYTES = 48     # R28: 32 bytes of 2-bit levels + 4 (m, s) fp16 pairs
 
 
 # ----------------------------------------------------------------------------
@@ -429,6 +447,62 @@ def kmeans_codebook(K: np.ndarray, mu: np.ndarray, init_idx, iters: int = KMEANS
         cent, counts = kmeans_update(x, assign, cent)
     code[num_sinks:] = assign
     return code, cent, counts
+
+
+# ----------------------------------------------------------------------------
+# 2-bit values  [SIKV §3, §4]  (R25-R28)
+# ----------------------------------------------------------------------------
+
+def quantize_values(V: np.ndarray) -> np.ndarray:
+    """Per-token 2-bit quantization of value rows (R25, R26, R28).
+
+    V holds stored values (exact in fp32), [N][D] with D = 128.  Returns the
+    48-byte rows, uint8 [N][48].
+    """
+    V32 = np.asarray(V, dtype=np.float64).astype(np.float32)
+    n, d = V32.shape
+    ng = d // V_GROUP
+    G = V32.reshape(n, ng, V_GROUP)
+    lo, hi = G.min(axis=2), G.max(axis=2)
+    step32 = (hi - lo) / np.float32(3)                     # two fp32 operations
+    m16, s16 = lo.astype(np.float16), step32.astype(np.float16)
+    m32, s32 = m16.astype(np.float32)[..., None], s16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (G - m32) / s32                                # fp32 subtraction, then fp32 division
+    level = np.where(s32 > 0, np.clip(np.rint(t), 0, 3), 0).astype(np.uint8).reshape(n, d // 4, 4)
+    out = np.zeros((n, V_ROW_BYTES), dtype=np.uint8)
+    out[:, :d // 4] = level[..., 0] | (level[..., 1] << 2) | (level[..., 2] << 4) | (level[..., 3] << 6)
+    out[:, d // 4:] = np.stack([m16, s16], axis=2).reshape(n, 2 * ng).view(np.uint8)
+    return out
+
+
+def dequantize_values(packed: np.ndarray, d: int = 128) -> np.ndarray:
+    """The values the quantized rows stand for: m + q s, float64 [N][D] (R25)."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    n = packed.shape[0]
+    ng = d // V_GROUP
+    b = packed[:, :d // 4]
+    level = np.stack([(b >> (2 * i)) & 3 for i in range(4)], axis=2).reshape(n, ng, V_GROUP).astype(np.float64)
+    ms = np.ascontiguousarray(packed[:, d // 4:d // 4 + 4 * ng]).view(np.float16).reshape(n, ng, 2).astype(np.float64)
+    return (ms[..., 0:1] + level * ms[..., 1:2]).reshape(n, d)
+
+
+def sparse_attention_qv(q_group, K, V, packed, mu, centroids, code, idx, num_sinks=DEFAULT_SINKS, scale=None):
+    """Sparse attention with 2-bit values for the selected tokens and
+    full-precision values for the sinks (R27); otherwise
+    :func:`sparse_attention`."""
+    Vmix = np.array(V, dtype=np.float64, copy=True)
+    s = min(num_sinks, Vmix.shape[0])
+    Vmix[s:] = dequantize_values(np.asarray(packed)[s:Vmix.shape[0]], Vmix.shape[1])
+    return sparse_attention(q_group, K, Vmix, mu, centroids, code, idx, num_sinks, scale)
+
+
+def decode_step_qv(q_group, K, V, packed, mu, centroids, code, k, num_sinks=DEFAULT_SINKS, scale=None):
+    """:func:`decode_step` with 2-bit values for the selected tokens (R27)."""
+    sc, cond = scores(q_group, mu, centroids, code, num_sinks)
+    idx = topk(sc, k, num_sinks)
+    out = sparse_attention_qv(q_group, K, V, packed, mu, centroids, code, idx, num_sinks, scale)
+    return out, idx, sc, cond
 
 
 def decode_step(q_group, K, V, mu, centroids, code, k, num_sinks=DEFAULT_SINKS, scale=None):

@@ -528,6 +528,88 @@ def check_kmeans_lloyd_invariants(o):
         assert prev is None or sse <= prev * (1 + 1e-6), (iters, sse, prev)
         prev = sse
 
+
+
+# --------------------------------------------------------------------------
+# 2-bit values (§3 and §4: accuracy kept with 2-bit quantization, the memory
+# saving of 2-bit KIVI; the scheme is a reading of this repository)
+# --------------------------------------------------------------------------
+
+def _golden_value_row():
+    g = _load("values_2bit_d128.json")
+    row = np.zeros(128, dtype=np.float32)
+    row[0:32] = np.tile(np.float32(g["row"]["group0"]), 8)
+    row[32:64] = g["row"]["group1"][0]
+    row[64:96] = np.tile(np.float32([-1.0, -1.0 / 3.0, 1.0 / 3.0, 1.0]), 8)
+    row[96:128] = np.tile(np.float32(g["row"]["group3"]), 4)
+    return g, row.astype(np.float64)
+
+
+def check_values_golden(o):
+    g, row = _golden_value_row()
+    packed = o.quantize_values(row[None])
+    assert packed.dtype == np.uint8 and packed.shape == (1, 48)
+    assert packed[0].tolist() == g["packed"]
+    back = o.dequantize_values(packed)[0]
+    rb = g["read_back"]
+    assert back[0:32].tolist() == list(map(float, rb["group0"])) * 8
+    assert back[32:64].tolist() == rb["group1"] * 32
+    assert back[64:96].tolist() == rb["group2"] * 8
+    assert back[96:128].tolist() == list(map(float, rb["group3"])) * 4
+
+
+def check_values_error_bound(o):
+    """Every value reads back within half a step of itself (plus the fp16
+    rounding of the group's minimum and step); a group's minimum reads back as
+    its fp16 minimum; values on an exact fp16 grid read back exactly."""
+    rng = np.random.default_rng(41)
+    V = (rng.standard_normal((300, 128)) * rng.uniform(0.1, 10.0, (300, 1))).astype(np.float32).astype(np.float64)
+    back = o.dequantize_values(o.quantize_values(V))
+    G = V.reshape(300, 4, 32)
+    lo, hi = G.min(axis=2), G.max(axis=2)
+    m16 = lo.astype(np.float16).astype(np.float64)
+    s = (hi - lo) / 3.0
+    s16 = s.astype(np.float16).astype(np.float64)
+    bound = s16 / 2 + np.abs(lo - m16) + 3 * np.abs(s - s16) + 1e-6 * np.abs(G).max(axis=2)
+    err = np.abs(back.reshape(300, 4, 32) - G).max(axis=2)
+    assert np.all(err <= bound)
+    amin = G.argmin(axis=2)
+    assert np.array_equal(np.take_along_axis(back.reshape(300, 4, 32), amin[..., None], 2)[..., 0], m16)
+    grid = rng.integers(0, 4, (50, 128)).astype(np.float64)
+    grid[:, ::32] = 0.0
+    grid[:, 1::32] = 3.0                                    # every group spans the four levels
+    Vg = -2.5 + 0.75 * grid
+    assert np.array_equal(o.dequantize_values(o.quantize_values(Vg)), Vg)
+
+
+def check_values_attention(o):
+    """Sinks keep full-precision values: with nothing selected the 2-bit
+    attention equals the full-precision one for any values; with values on
+    an exact grid it equals it for any selection; otherwise the outputs differ
+    by at most the largest read-back error (softmax weights form a convex
+    combination)."""
+    rng = np.random.default_rng(43)
+    s, n, d = 4, 60, 128
+    K = rng.standard_normal((n, d))
+    V = (rng.standard_normal((n, d)) * 3).astype(np.float32).astype(np.float64)
+    q = rng.standard_normal((2, d))
+    mu, code, cent, _ = o.encode_keys(K, s)
+    packed = o.quantize_values(V)
+    none = np.zeros(0, dtype=np.int64)
+    assert np.allclose(o.sparse_attention_qv(q, K, V, packed, mu, cent, code, none, s),
+                       o.sparse_attention(q, K, V, mu, cent, code, none, s), rtol=0, atol=1e-12)
+    idx = np.arange(s, n, 3)
+    full = o.sparse_attention(q, K, V, mu, cent, code, idx, s)
+    qv = o.sparse_attention_qv(q, K, V, packed, mu, cent, code, idx, s)
+    worst = np.abs(o.dequantize_values(packed) - V)[idx].max()
+    assert np.all(np.abs(qv - full) <= worst + 1e-12) and not np.allclose(qv, full, rtol=0, atol=1e-9)
+    grid = rng.integers(0, 4, (n, d)).astype(np.float64)
+    grid[:, ::32] = 0.0
+    grid[:, 1::32] = 3.0
+    Vg = 1.25 + 0.5 * grid
+    assert np.allclose(o.sparse_attention_qv(q, K, Vg, o.quantize_values(Vg), mu, cent, code, idx, s),
+                       o.sparse_attention(q, K, Vg, mu, cent, code, idx, s), rtol=0, atol=1e-12)
+
 ALL_CHECKS = [
     check_exact_sum, check_round_to_f32, check_channel_mean, check_sign_codes_golden,
     check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
@@ -536,5 +618,5 @@ ALL_CHECKS = [
     check_attention_invariants, check_needle_recall, check_append_by_construction, check_append_golden,
     check_dense_scores_equal_lut_scores_when_exact, check_dense_attention,
     check_kmeans_golden, check_kmeans_update_exact, check_kmeans_matches_sklearn,
-    check_kmeans_lloyd_invariants,
+    check_kmeans_lloyd_invariants, check_values_golden, check_values_error_bound, check_values_attention,
 ]

@@ -1,5 +1,6 @@
 """The CPU oracle against hand-worked examples, closed forms and invariants."""
 
+import builtins
 import copy
 import types
 
@@ -18,6 +19,7 @@ def test_oracle_pin(check):
 def _mutant(**overrides):
     m = types.ModuleType("oracle_mutant")
     m.__dict__.update({k: v for k, v in vars(oracle).items() if not k.startswith("__")})
+    m.__dict__["__builtins__"] = builtins          # the rebound functions look builtins up here
     m.__dict__.update(overrides)
     # rebind module-level helpers so composite functions use the mutated pieces
     for name, fn in list(vars(oracle).items()):
@@ -134,6 +136,32 @@ def _mut_kmeans_one_short(K, mu, init_idx, iters=20, num_sinks=64):
     return oracle.kmeans_codebook(K, mu, init_idx, max(iters - 1, 1), num_sinks)
 
 
+def _mut_values(level_fn=None, step_div=3.0, group=32, msb_first=False):
+    def quantize(V):
+        V32 = np.asarray(V, dtype=np.float64).astype(np.float32)
+        n, d = V32.shape
+        G = V32.reshape(n, d // group, group)
+        lo, hi = G.min(axis=2), G.max(axis=2)
+        m16, s16 = lo.astype(np.float16), ((hi - lo) / np.float32(step_div)).astype(np.float16)
+        m32, s32 = m16.astype(np.float32)[..., None], s16.astype(np.float32)[..., None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            t = (G - m32) / s32
+        r = level_fn(t) if level_fn else np.rint(t)
+        lv = np.where(s32 > 0, np.clip(r, 0, 3), 0).astype(np.uint8).reshape(n, d // 4, 4)
+        out = np.zeros((n, 48), dtype=np.uint8)
+        sh = [6, 4, 2, 0] if msb_first else [0, 2, 4, 6]
+        out[:, :d // 4] = (lv[..., 0] << sh[0]) | (lv[..., 1] << sh[1]) | (lv[..., 2] << sh[2]) | (lv[..., 3] << sh[3])
+        prm = np.stack([m16, s16], axis=2).reshape(n, -1)[:, :8]
+        out[:, d // 4:] = prm.view(np.uint8)
+        return out
+    return quantize
+
+
+def _mut_values_sinks_quantized(q_group, K, V, packed, mu, centroids, code, idx, num_sinks=64, scale=None):
+    Vq = oracle.dequantize_values(np.asarray(packed)[:np.asarray(V).shape[0]], np.asarray(V).shape[1])
+    return oracle.sparse_attention(q_group, K, Vq, mu, centroids, code, idx, num_sinks, scale)
+
+
 MUTATIONS = {
     "strict-greater": dict(sign_codes=_mut_codes_strict),
     "msb-first-bits": dict(sign_codes=_mut_codes_msb_first),
@@ -153,6 +181,11 @@ MUTATIONS = {
     "kmeans-no-mean-normalization": dict(kmeans_points=_mut_kmeans_no_mu),
     "kmeans-clusters-sinks": dict(kmeans_codebook=_mut_kmeans_with_sinks),
     "kmeans-one-iteration-short": dict(kmeans_codebook=_mut_kmeans_one_short),
+    "values-round-half-up": dict(quantize_values=_mut_values(level_fn=lambda t: np.floor(t + np.float32(0.5)))),
+    "values-step-over-4": dict(quantize_values=_mut_values(step_div=4.0)),
+    "values-levels-msb-first": dict(quantize_values=_mut_values(msb_first=True)),
+    "values-groups-of-16": dict(quantize_values=_mut_values(group=16)),
+    "values-sinks-quantized": dict(sparse_attention_qv=_mut_values_sinks_quantized),
 }
 
 
