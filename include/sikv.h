@@ -129,6 +129,7 @@ SIKV_API size_t sikv_decode_host_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_append_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_dense_attn_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_kmeans_workspace_size(const sikv_params *p);
+SIKV_API size_t sikv_quantize_values_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
  * (0 on bad params). */
@@ -269,6 +270,41 @@ SIKV_API sikv_status sikv_dense_score(const sikv_params *p, const void *q, const
 SIKV_API sikv_status sikv_dense_attn(const sikv_params *p, const void *q, const void *K, const void *V,
                                      const int32_t *seq_lens, void *out, void *workspace, size_t workspace_bytes,
                                      sikv_stream_t stream);
+
+/*
+ * 2-bit values -- the operating point the pages report accuracy for with
+ * 2-bit quantization and a memory saving equal to 2-bit KIVI's [SIKV 3, 4];
+ * the scheme is not given there.  This is KIVI's per-token value
+ * quantization, read as:
+ *   each token's row of V is cut into 4 groups of 32 channels; a group keeps
+ *   m16 = fp16(min) and s16 = fp16(fl32(fl32(max - min) / 3)) (round to
+ *   nearest even), and each value the level
+ *       q = clamp(rint(fl32(fl32(v - m16) / s16)), 0, 3)   (ties to even; 0 when s16 = 0)
+ *   that reads back as m16 + q * s16.  Values must lie in the fp16 range.
+ * Row layout (48 bytes, the vq arrays below): 32 bytes of levels, dimension d
+ * in bits 2 (d mod 4) of byte d / 4 (LSB first), then (m16, s16) of groups
+ * 0..3, little-endian.  vq is device u8 [B][Hkv][Nmax][48], 16-byte aligned.
+ *
+ * sikv_quantize_values: rows t in [0, N_b) of vq from V (dtype
+ * [B][Hkv][Nmax][D]); other rows are not written.  An invalid seq_lens[b]
+ * sets SIKV_DEVERR_SEQ_LEN and skips the sequence.  workspace:
+ * sikv_quantize_values_workspace_size() bytes (the status header).
+ *
+ * sikv_decode_qv / sikv_sparse_attn_qv: sikv_decode / sikv_sparse_attn with
+ * the selected tokens' values read from vq; the sinks keep reading their
+ * full-precision rows of V.  Arguments, workspaces and errors as there.
+ */
+SIKV_API sikv_status sikv_quantize_values(const sikv_params *p, const void *V, const int32_t *seq_lens, uint8_t *vq,
+                                          void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+SIKV_API sikv_status sikv_decode_qv(const sikv_params *p, const void *q, const void *K, const void *V,
+                                    const uint8_t *vq, const uint8_t *codes, const float *codebook, const float *mu,
+                                    const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
+                                    float *scores_out, void *workspace, size_t workspace_bytes, sikv_stream_t stream);
+SIKV_API sikv_status sikv_sparse_attn_qv(const sikv_params *p, const void *q, const void *K, const void *V,
+                                         const uint8_t *vq, const uint8_t *codes, const float *codebook,
+                                         const float *mu, const int32_t *idx, const int32_t *k_per_seq,
+                                         const int32_t *seq_lens, void *out, void *workspace, size_t workspace_bytes,
+                                         sikv_stream_t stream);
 
 /*
  * sikv_kmeans_codebook -- comparison baseline, not the method: the iterative

@@ -19,7 +19,7 @@ from ._binding import (EXPORTED, SIKV_DEVERR_APPEND, SIKV_DEVERR_INDEX, SIKV_DEV
                        SIKV_DEVERR_TOPK, SIKV_DTYPE_BF16, SIKV_DTYPE_F32, DecodeHostPlan, Params, SikvError,
                        Workspace, default_scale, lib, library_path, make_params, sikv_append_codes, sikv_decode,
                        sikv_decode_host, sikv_dense_attn, sikv_dense_score, sikv_encode_keys, sikv_kmeans_codebook,
-                       sikv_score,
+                       sikv_score, sikv_quantize_values, sikv_decode_qv, sikv_sparse_attn_qv, VQ_ROW_BYTES,
                        sikv_sparse_attn, sikv_topk, version, workspace_size)
 
 
@@ -52,6 +52,7 @@ class SikvCache:
         self.counts = torch.empty((B, H, D // 4, 16), dtype=torch.int32, device=dev)
         self.ws_encode = Workspace(workspace_size("encode", p), dev)
         self.ws_decode = Workspace(workspace_size("decode", p), dev)
+        self.vq = None            # 2-bit value rows, made by quantize_values()
 
     def encode(self, stream=None):
         sikv_encode_keys(self.p, self.K, self.seq_lens, self.mu, self.codes, self.codebook, self.counts,
@@ -63,6 +64,23 @@ class SikvCache:
         ``seq_lens`` afterwards to make them visible to ``decode``."""
         sikv_append_codes(self.p, self.K, start, count, self.mu, self.codes, workspace=self.ws_encode,
                           stream=stream)
+
+    def quantize_values(self, stream=None):
+        """2-bit rows of V for the selected tokens' values (sinks keep V);
+        ``decode_qv`` reads them."""
+        if self.vq is None:
+            p = self.p
+            self.vq = torch.empty((p.batch, p.num_kv_heads, p.max_seq_len, VQ_ROW_BYTES), dtype=torch.uint8,
+                                  device=self.K.device)
+        sikv_quantize_values(self.p, self.V, self.seq_lens, self.vq, workspace=self.ws_encode, stream=stream)
+
+    def decode_qv(self, q, k_per_seq, out=None, idx_out=None, scores_out=None, stream=None):
+        """One decode step reading the selected tokens' values from the 2-bit rows."""
+        if out is None:
+            out = torch.empty_like(q)
+        sikv_decode_qv(self.p, q, self.K, self.V, self.vq, self.codes, self.codebook, self.mu, self.seq_lens,
+                       k_per_seq, out, idx_out=idx_out, scores_out=scores_out, workspace=self.ws_decode, stream=stream)
+        return out
 
     def decode(self, q, k_per_seq, out=None, idx_out=None, scores_out=None, stream=None):
         if out is None:

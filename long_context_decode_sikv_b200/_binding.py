@@ -36,7 +36,10 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
             "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
             "sikv_append_workspace_size", "sikv_append_codes", "sikv_dense_attn_workspace_size",
-            "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_workspace_size", "sikv_kmeans_codebook")
+            "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_workspace_size", "sikv_kmeans_codebook",
+            "sikv_quantize_values_workspace_size", "sikv_quantize_values", "sikv_decode_qv", "sikv_sparse_attn_qv")
+
+VQ_ROW_BYTES = 48     # a token's 2-bit value row: 32 bytes of levels + 4 (min, step) fp16 pairs
 
 
 class SikvError(RuntimeError):
@@ -100,7 +103,8 @@ def lib() -> ctypes.CDLL:
         for n in ("sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
                   "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size",
                   "sikv_decode_host_workspace_size", "sikv_append_workspace_size",
-                  "sikv_dense_attn_workspace_size", "sikv_kmeans_workspace_size"):
+                  "sikv_dense_attn_workspace_size", "sikv_kmeans_workspace_size",
+                  "sikv_quantize_values_workspace_size"):
             getattr(L, n).restype = sz
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
@@ -115,9 +119,13 @@ def lib() -> ctypes.CDLL:
         L.sikv_dense_score.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_dense_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_kmeans_codebook.argtypes = [pp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+        L.sikv_quantize_values.argtypes = [pp, vp, vp, vp, vp, sz, vp]
+        L.sikv_decode_qv.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_sparse_attn_qv.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
                   "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes",
-                  "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_codebook"):
+                  "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_codebook", "sikv_quantize_values",
+                  "sikv_decode_qv", "sikv_sparse_attn_qv"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -323,6 +331,56 @@ def sikv_decode(p: Params, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, ou
             _ptr(scores_out, "scores_out", torch.float32, (B, H, N), dev, optional=True))
     ws = _ws("decode", p, workspace, dev, stream)
     _check(lib().sikv_decode(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_decode")
+    return ws
+
+
+def sikv_quantize_values(p: Params, V, seq_lens, vq, workspace=None, stream=None):
+    """2-bit value rows vq [B][Hkv][Nmax][48] (uint8) of V's rows [0, N_b)."""
+    dev = V.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(vq, "vq", torch.uint8, (B, H, N, VQ_ROW_BYTES), dev))
+    ws = _ws("quantize_values", p, workspace, dev, stream)
+    _check(lib().sikv_quantize_values(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)),
+           "sikv_quantize_values")
+    return ws
+
+
+def sikv_sparse_attn_qv(p: Params, q, K, V, vq, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
+                        workspace=None, stream=None):
+    """:func:`sikv_sparse_attn` with the selected tokens' values read from the 2-bit rows vq."""
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(vq, "vq", torch.uint8, (B, H, N, VQ_ROW_BYTES), dev),
+            _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev),
+            _ptr(idx, "idx", torch.int32, (B, H, p.max_topk), dev, optional=p.max_topk == 0),
+            _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(out, "out", p.torch_dtype, (B, p.num_q_heads, D), dev))
+    ws = _ws("sparse_attn", p, workspace, dev, stream)
+    _check(lib().sikv_sparse_attn_qv(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)),
+           "sikv_sparse_attn_qv")
+    return ws
+
+
+def sikv_decode_qv(p: Params, q, K, V, vq, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out=None,
+                   scores_out=None, workspace=None, stream=None):
+    """:func:`sikv_decode` with the selected tokens' values read from the 2-bit rows vq."""
+    dev = q.device
+    B, H, N, D = p.batch, p.num_kv_heads, p.max_seq_len, p.head_dim
+    args = (_ptr(q, "q", p.torch_dtype, (B, p.num_q_heads, D), dev), _ptr(K, "K", p.torch_dtype, (B, H, N, D), dev),
+            _ptr(V, "V", p.torch_dtype, (B, H, N, D), dev), _ptr(vq, "vq", torch.uint8, (B, H, N, VQ_ROW_BYTES), dev),
+            _ptr(codes, "codes", torch.uint8, (B, H, N, D // 8), dev),
+            _ptr(codebook, "codebook", torch.float32, (B, H, D // 4, 16, 4), dev),
+            _ptr(mu, "mu", torch.float32, (B, H, D), dev), _ptr(seq_lens, "seq_lens", torch.int32, (B,), dev),
+            _ptr(k_per_seq, "k_per_seq", torch.int32, (B,), dev),
+            _ptr(out, "out", p.torch_dtype, (B, p.num_q_heads, D), dev),
+            _ptr(idx_out, "idx_out", torch.int32, (B, H, p.max_topk), dev, optional=True),
+            _ptr(scores_out, "scores_out", torch.float32, (B, H, N), dev, optional=True))
+    ws = _ws("decode", p, workspace, dev, stream)
+    _check(lib().sikv_decode_qv(ctypes.byref(p), *args, ws.ptr, ws.nbytes, _stream(stream, dev)), "sikv_decode_qv")
     return ws
 
 

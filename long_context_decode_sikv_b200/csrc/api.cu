@@ -116,10 +116,10 @@ void *device_view(const void *host) {
 
 // One decode step on device buffers (arguments checked here, except q and
 // out, which the callers check).
-sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, const void *V, const uint8_t *codes,
-                        const float *codebook, const float *mu, const int32_t *seq_lens, const int32_t *k_per_seq,
-                        void *out, int32_t *idx_out, float *scores_out, void *workspace, size_t workspace_bytes,
-                        cudaStream_t s) {
+sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, const void *V, const uint8_t *vq,
+                        const uint8_t *codes, const float *codebook, const float *mu, const int32_t *seq_lens,
+                        const int32_t *k_per_seq, void *out, int32_t *idx_out, float *scores_out, void *workspace,
+                        size_t workspace_bytes, cudaStream_t s) {
     const sikv_params *p = &pp;
     SIKV_REQUIRE_PTR(K);
     SIKV_REQUIRE_PTR(V);
@@ -132,26 +132,29 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
     SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
     char *ws = static_cast<char *>(workspace);
     int32_t *status = reinterpret_cast<int32_t *>(ws);
-    const FusedPlan plan = fused_plan(*p);
+    const bool qv = vq != nullptr;
+    const FusedPlan plan = fused_plan(*p, qv);
     if (plan.ok)
-        return launch_decode_fused(*p, plan, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
+        return launch_decode_fused(*p, plan, q, K, V, vq, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
                                    scores_out, ws, L.fused, status, s);
     // Too many segments for one co-resident launch: run the single-launch
     // kernel on sub-batches of sequences that fit, one after the other on the
     // stream (each launch leaves the coordination state zeroed for the next).
-    const int bsub = fused_sub_batch(*p);
+    const int bsub = fused_sub_batch(*p, qv);
     if (bsub > 0) {
         const size_t eb = p->dtype == SIKV_DTYPE_F32 ? 4 : 2;
         const size_t hq = p->num_q_heads, hkv = p->num_kv_heads, nmax = p->max_seq_len, d = p->head_dim;
         for (int b0 = 0; b0 < p->batch; b0 += bsub) {
             sikv_params ps = *p;
             ps.batch = std::min(bsub, p->batch - b0);
-            const FusedPlan pl = fused_plan(ps);
+            const FusedPlan pl = fused_plan(ps, qv);
             if (!pl.ok) return SIKV_ERR_UNSUPPORTED;      // cannot happen: fused_sub_batch checked it
             const size_t bq = static_cast<size_t>(b0) * hq * d * eb, bkv = static_cast<size_t>(b0) * hkv * nmax * d * eb;
             SIKV_TRY(launch_decode_fused(
                 ps, pl, static_cast<const char *>(q) + bq, static_cast<const char *>(K) + bkv,
-                static_cast<const char *>(V) + bkv, codes + static_cast<size_t>(b0) * hkv * nmax * (d / 8),
+                static_cast<const char *>(V) + bkv,
+                qv ? vq + static_cast<size_t>(b0) * hkv * nmax * kVqRowBytes : nullptr,
+                codes + static_cast<size_t>(b0) * hkv * nmax * (d / 8),
                 codebook + static_cast<size_t>(b0) * hkv * kSubspaces * kClusters * 4,
                 mu + static_cast<size_t>(b0) * hkv * d, seq_lens + b0, k_per_seq + b0, static_cast<char *>(out) + bq,
                 idx_out ? idx_out + static_cast<size_t>(b0) * hkv * (p->max_topk > 0 ? p->max_topk : 0) : nullptr,
@@ -163,7 +166,7 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
     int32_t *ix = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     SIKV_TRY(launch_score(*p, q, codes, codebook, mu, seq_lens, sc, status, s));
     if (p->max_topk > 0) SIKV_TRY(launch_topk(*p, sc, seq_lens, k_per_seq, ix, status, s));
-    return launch_sparse_attn(*p, q, K, V, codes, codebook, mu, ix, k_per_seq, seq_lens, out, ws, L.attn,
+    return launch_sparse_attn(*p, q, K, V, vq, codes, codebook, mu, ix, k_per_seq, seq_lens, out, ws, L.attn,
                               status, s);
 }
 
@@ -377,9 +380,47 @@ sikv_status sikv_sparse_attn(const sikv_params *p, const void *q, const void *K,
     SIKV_REQUIRE_PTR4(seq_lens);
     SIKV_REQUIRE_PTR(out);
     SIKV_TRY(check_ws(workspace, workspace_bytes, attn_layout(*p, kHeaderBytes).total));
-    return launch_sparse_attn(*p, q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
+    return launch_sparse_attn(*p, q, K, V, nullptr, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
                               static_cast<char *>(workspace), kHeaderBytes, static_cast<int32_t *>(workspace),
                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+sikv_status sikv_sparse_attn_qv(const sikv_params *p, const void *q, const void *K, const void *V, const uint8_t *vq,
+                                const uint8_t *codes, const float *codebook, const float *mu, const int32_t *idx,
+                                const int32_t *k_per_seq, const int32_t *seq_lens, void *out, void *workspace,
+                                size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(q);
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR(V);
+    SIKV_REQUIRE_PTR(vq);
+    SIKV_REQUIRE_PTR(codes);
+    SIKV_REQUIRE_PTR(codebook);
+    SIKV_REQUIRE_PTR(mu);
+    if (p->max_topk > 0) SIKV_REQUIRE_PTR4(idx);
+    SIKV_REQUIRE_PTR4(k_per_seq);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR(out);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, attn_layout(*p, kHeaderBytes).total));
+    return launch_sparse_attn(*p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
+                              static_cast<char *>(workspace), kHeaderBytes, static_cast<int32_t *>(workspace),
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sikv_quantize_values_workspace_size(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return kHeaderBytes;
+}
+
+sikv_status sikv_quantize_values(const sikv_params *p, const void *V, const int32_t *seq_lens, uint8_t *vq,
+                                 void *workspace, size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(V);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR(vq);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, kHeaderBytes));
+    return sikv::launch_quantize_values(*p, V, seq_lens, vq, static_cast<int32_t *>(workspace),
+                                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 sikv_status sikv_decode(const sikv_params *p, const void *q, const void *K, const void *V,
@@ -391,7 +432,21 @@ sikv_status sikv_decode(const sikv_params *p, const void *q, const void *K, cons
     SIKV_REQUIRE_PTR(out);
     if (idx_out) SIKV_REQUIRE_PTR4(idx_out);
     if (scores_out) SIKV_REQUIRE_PTR4(scores_out);
-    return sikv::decode_step(*p, q, K, V, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out, scores_out,
+    return sikv::decode_step(*p, q, K, V, nullptr, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
+                             scores_out, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sikv_status sikv_decode_qv(const sikv_params *p, const void *q, const void *K, const void *V, const uint8_t *vq,
+                           const uint8_t *codes, const float *codebook, const float *mu, const int32_t *seq_lens,
+                           const int32_t *k_per_seq, void *out, int32_t *idx_out, float *scores_out, void *workspace,
+                           size_t workspace_bytes, sikv_stream_t stream) {
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(q);
+    SIKV_REQUIRE_PTR(out);
+    SIKV_REQUIRE_PTR(vq);
+    if (idx_out) SIKV_REQUIRE_PTR4(idx_out);
+    if (scores_out) SIKV_REQUIRE_PTR4(scores_out);
+    return sikv::decode_step(*p, q, K, V, vq, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out, scores_out,
                              workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -416,7 +471,7 @@ sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const voi
         if (cudaMemcpyAsync(ws + H.q, q_host, H.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return SIKV_ERR_CUDA;
         q_dev = ws + H.q;
     }
-    SIKV_TRY(sikv::decode_step(*p, q_dev, K, V, codes, codebook, mu, seq_lens, k_per_seq,
+    SIKV_TRY(sikv::decode_step(*p, q_dev, K, V, nullptr, codes, codebook, mu, seq_lens, k_per_seq,
                                out_dev ? out_dev : ws + H.out, nullptr, nullptr, workspace, decode_total, s));
     if (!out_dev &&
         cudaMemcpyAsync(out_host, ws + H.out, H.bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -35,10 +35,10 @@ struct AttnSmem {
     alignas(16) float red[kAttnWarps][G][kHeadDim];   // written with float4 stores
 };
 
-template <int DT, int G>
+template <int DT, int G, bool VQ>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_partial_kernel(const void *__restrict__ q, const void *__restrict__ K, const void *__restrict__ V,
-                    const uint8_t *__restrict__ codes, const float *__restrict__ codebook,
+                    const uint8_t *__restrict__ vq, const uint8_t *__restrict__ codes, const float *__restrict__ codebook,
                     const float *__restrict__ mu, const int32_t *__restrict__ idx,
                     const int32_t *__restrict__ k_per_seq, const int32_t *__restrict__ seq_lens,
                     int hq, int hkv, int nmax, int num_sinks, int kmax, int nsplit, float scale,
@@ -186,8 +186,12 @@ attn_partial_kernel(const void *__restrict__ q, const void *__restrict__ K, cons
         for (int u = 0; u < kVRows; ++u) {
             const int i = i0 + u * kAttnWarps;
             const int t = (i < n_here) ? sh.tok[i] : -1;
-            v[u] = (t >= 0) ? load4<DT>(static_cast<const char *>(V) + (kv_seg + t) * kHeadDim * EB, lane * 4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < 0)
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            else if (VQ && t >= num_sinks)   // a selected token's 2-bit row (sinks read V)
+                v[u] = vq_decode4(vq + (kv_seg + t) * kVqRowBytes, lane);
+            else
+                v[u] = load4<DT>(static_cast<const char *>(V) + (kv_seg + t) * kHeadDim * EB, lane * 4);
         }
 #pragma unroll
         for (int u = 0; u < kVRows; ++u) {
@@ -251,18 +255,18 @@ attn_combine_kernel(const float *__restrict__ part_o, const float2 *__restrict__
         static_cast<unsigned short *>(out)[orow] = static_cast<unsigned short>(f32_to_bf16_bits(r));
 }
 
-template <int DT, int G>
-sikv_status launch_partial(const sikv_params &p, const void *q, const void *K, const void *V,
+template <int DT, int G, bool VQ>
+sikv_status launch_partial(const sikv_params &p, const void *q, const void *K, const void *V, const uint8_t *vq,
                            const uint8_t *codes, const float *codebook, const float *mu,
                            const int32_t *idx, const int32_t *k_per_seq, const int32_t *seq_lens,
                            const AttnLayout &L, char *ws, float scale, int32_t *status,
                            cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem<G>);
-    auto kern = attn_partial_kernel<DT, G>;
+    auto kern = attn_partial_kernel<DT, G, VQ>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SIKV_ERR_CUDA;
     const dim3 grid(L.nsplit, p.batch * p.num_kv_heads);
-    kern<<<grid, kAttnThreads, smem, stream>>>(q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens,
+    kern<<<grid, kAttnThreads, smem, stream>>>(q, K, V, vq, codes, codebook, mu, idx, k_per_seq, seq_lens,
                                                p.num_q_heads, p.num_kv_heads, p.max_seq_len, p.num_sinks,
                                                p.max_topk, L.nsplit, scale,
                                                reinterpret_cast<float *>(ws + L.part_o),
@@ -270,15 +274,15 @@ sikv_status launch_partial(const sikv_params &p, const void *q, const void *K, c
     return SIKV_OK;
 }
 
-template <int DT>
+template <int DT, bool VQ>
 sikv_status dispatch_group(int group, const sikv_params &p, const void *q, const void *K, const void *V,
-                           const uint8_t *codes, const float *codebook, const float *mu,
+                           const uint8_t *vq, const uint8_t *codes, const float *codebook, const float *mu,
                            const int32_t *idx, const int32_t *k_per_seq, const int32_t *seq_lens,
                            const AttnLayout &L, char *ws, float scale, int32_t *status,
                            cudaStream_t stream) {
 #define SIKV_G(NG) \
     case NG:       \
-        return launch_partial<DT, NG>(p, q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens, L, ws, scale, status, stream)
+        return launch_partial<DT, NG, VQ>(p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq, seq_lens, L, ws, scale, status, stream)
     switch (group) {
         SIKV_G(1);
         SIKV_G(2);
@@ -313,7 +317,7 @@ AttnLayout attn_layout(const sikv_params &p, size_t base) {
 }
 
 sikv_status launch_sparse_attn(const sikv_params &p, const void *q, const void *K, const void *V,
-                               const uint8_t *codes, const float *codebook, const float *mu,
+                               const uint8_t *vq, const uint8_t *codes, const float *codebook, const float *mu,
                                const int32_t *idx, const int32_t *k_per_seq,
                                const int32_t *seq_lens, void *out, char *ws, size_t attn_base,
                                int32_t *status, cudaStream_t stream) {
@@ -322,11 +326,15 @@ sikv_status launch_sparse_attn(const sikv_params &p, const void *q, const void *
     const float scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf(static_cast<float>(p.head_dim));
     sikv_status st;
     if (p.dtype == SIKV_DTYPE_BF16)
-        st = dispatch_group<SIKV_DTYPE_BF16>(group, p, q, K, V, codes, codebook, mu, idx, k_per_seq,
-                                             seq_lens, L, ws, scale, status, stream);
+        st = vq ? dispatch_group<SIKV_DTYPE_BF16, true>(group, p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq,
+                                                        seq_lens, L, ws, scale, status, stream)
+                : dispatch_group<SIKV_DTYPE_BF16, false>(group, p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq,
+                                                         seq_lens, L, ws, scale, status, stream);
     else
-        st = dispatch_group<SIKV_DTYPE_F32>(group, p, q, K, V, codes, codebook, mu, idx, k_per_seq,
-                                            seq_lens, L, ws, scale, status, stream);
+        st = vq ? dispatch_group<SIKV_DTYPE_F32, true>(group, p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq,
+                                                       seq_lens, L, ws, scale, status, stream)
+                : dispatch_group<SIKV_DTYPE_F32, false>(group, p, q, K, V, vq, codes, codebook, mu, idx, k_per_seq,
+                                                        seq_lens, L, ws, scale, status, stream);
     if (st != SIKV_OK) return st;
     const dim3 grid(group, p.batch * p.num_kv_heads);
     const float *po = reinterpret_cast<const float *>(ws + L.part_o);

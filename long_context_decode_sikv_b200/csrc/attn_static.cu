@@ -80,7 +80,7 @@ extern "C" sikv_status sikv_sparse_attn_static(const sikv_params *p, const void 
     // The array keeps the previous call's contents: only the status word has
     // to start at zero (every partial the kernels read is written first).
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return SIKV_ERR_CUDA;
-    const sikv_status st = launch_sparse_attn(*p, q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
+    const sikv_status st = launch_sparse_attn(*p, q, K, V, nullptr, codes, codebook, mu, idx, k_per_seq, seq_lens, out,
                                               scratch, kHeaderBytes, status, s);
     if (st != SIKV_OK) return st;
     if (device_flags &&

@@ -57,6 +57,7 @@ constexpr int kFRow = 256;               // tokens per row scan of a warp (32 la
 
 struct FusedArgs {
     const void *q, *K, *V;
+    const uint8_t *vq;    // 2-bit value rows of the selected tokens (VQ kernels only)
     const uint8_t *codes;
     const float *codebook, *mu;
     const int32_t *seq_lens, *k_per_seq;
@@ -381,18 +382,18 @@ __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wai
 
 // Value rows staged by a warp: two halves of its buffer, so that one half
 // is consumed while the other is in flight.
-template <int DT>
+template <int DT, bool VQ>
 struct VStage {
-    static constexpr int kRowBytes = kHeadDim * ElemBytes<DT>::value;
-    static constexpr int kHalf = kFVBytes / kRowBytes / 2;  // 8 (bf16) or 4 (fp32) rows
+    static constexpr int kRowBytes = VQ ? kVqRowBytes : kHeadDim * ElemBytes<DT>::value;
+    static constexpr int kHalf = VQ ? 16 : kFVBytes / kRowBytes / 2;  // 16 (2-bit), 8 (bf16) or 4 (fp32) rows
 };
 
 // Starts copying the value rows of tokens tok[j0 .. j0 + n) into vb (row j
 // at j * kRowBytes), 16 bytes per copy, all in flight at once.
-template <int DT>
+template <int DT, bool VQ>
 __device__ __forceinline__ void warp_stage_v(char *vb, const int32_t *tok, int j0, int n, const char *vseg,
                                              int lane) {
-    constexpr int kRowBytes = VStage<DT>::kRowBytes, kChunks = kRowBytes / 16;
+    constexpr int kRowBytes = VStage<DT, VQ>::kRowBytes, kChunks = kRowBytes / 16;
 #pragma unroll 1
     for (int i = lane; i < n * kChunks; i += 32) {
         const int j = i / kChunks, cc = i % kChunks;
@@ -402,15 +403,17 @@ __device__ __forceinline__ void warp_stage_v(char *vb, const int32_t *tok, int j
 }
 
 // o += sum over the staged rows j < n of pr_{j0+j} V[row j]; lane l takes
-// columns 4l..4l+3.
-template <int DT, int GM>
+// columns 4l..4l+3 (a 2-bit row is read back as min + level * step).
+template <int DT, int GM, bool VQ>
 __device__ __forceinline__ void warp_fma_v(WarpSoftmax<GM> &s, const char *vb, const float (&pr)[GM], int j0, int n,
                                            int lane) {
-    constexpr int kRowBytes = VStage<DT>::kRowBytes;
+    constexpr int kRowBytes = VStage<DT, VQ>::kRowBytes;
 #pragma unroll 2
     for (int j = 0; j < n; ++j) {
         float4 vv;
-        if (DT == SIKV_DTYPE_BF16) {
+        if (VQ) {
+            vv = vq_decode4(reinterpret_cast<const uint8_t *>(vb + j * kRowBytes), lane);
+        } else if (DT == SIKV_DTYPE_BF16) {
             const uint2 w = *reinterpret_cast<const uint2 *>(vb + j * kRowBytes + 8 * lane);
             vv = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
         } else {
@@ -451,7 +454,7 @@ __device__ __noinline__ uint32_t refine_by_radix(const uint2 *cand, int ncand, u
     return before;
 }
 
-template <int DT, int GM>
+template <int DT, int GM, bool VQ>
 __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     constexpr int EB = ElemBytes<DT>::value;
     extern __shared__ __align__(16) unsigned char fused_smem[];
@@ -636,6 +639,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     int bstar = kFBins;              // nothing selected when k == 0
     uint32_t above_bstar = 0, n_sure = 0;
     const char *vseg = static_cast<const char *>(a.V) + kv_seg * kHeadDim * EB;
+    // value rows of the selected tokens: V itself, or its 2-bit rows (sinks
+    // always read V)
+    const char *vsel = VQ ? reinterpret_cast<const char *>(a.vq) + kv_seg * kVqRowBytes : vseg;
     uint32_t *pend = sh.hist;                                        // free: the local histogram is published
     // each warp's direct list of attended tokens (kFWarpList entries)
     int32_t *wlist = reinterpret_cast<int32_t *>(sh.hist) + 2 * kFPend + kFWarpList * warp;
@@ -682,8 +688,13 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
             const int t = t0 + (warp + kFW * (bit >> 3)) * kFRow + 8 * lane + (bit & 7);
             if (pos < static_cast<uint32_t>(kFWarpList)) wlist[pos] = t;
             prefetch_l2(crow + t);
-            prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
-            if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+            if (VQ) {                              // a 48-byte row may straddle two lines
+                prefetch_l2(vsel + static_cast<size_t>(t) * kVqRowBytes);
+                prefetch_l2(vsel + static_cast<size_t>(t) * kVqRowBytes + kVqRowBytes - 1);
+            } else {
+                prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB);
+                if (EB * kHeadDim > 128) prefetch_l2(vseg + static_cast<size_t>(t) * kHeadDim * EB + 128);
+            }
         }
         for (unsigned long long mm = emask; mm; mm &= mm - 1) {
             const int bit = __ffsll(static_cast<long long>(mm)) - 1;
@@ -927,10 +938,10 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                 // then each half-buffer is refilled as soon as it is consumed
                 // (one copy group per half, so waiting for "all but one group"
                 // always means the half about to be read)
-                constexpr int kVH = VStage<DT>::kHalf, kHB = kVH * VStage<DT>::kRowBytes;
-                warp_stage_v<DT>(vb, tok, 0, min(nb, kVH), vseg, lane);
+                constexpr int kVH = VStage<DT, VQ>::kHalf, kHB = kVH * VStage<DT, VQ>::kRowBytes;
+                warp_stage_v<DT, VQ>(vb, tok, 0, min(nb, kVH), vsel, lane);
                 cp_async_commit();
-                warp_stage_v<DT>(vb + kHB, tok, kVH, max(0, min(nb - kVH, kVH)), vseg, lane);
+                warp_stage_v<DT, VQ>(vb + kHB, tok, kVH, max(0, min(nb - kVH, kVH)), vsel, lane);
                 cp_async_commit();
                 float lg[GM];
 #pragma unroll
@@ -962,9 +973,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                     char *hb = vb + half * kHB;
                     cp_async_wait_one();
                     __syncwarp();
-                    warp_fma_v<DT, GM>(ws, hb, lg, j0, min(kVH, nb - j0), lane);
+                    warp_fma_v<DT, GM, VQ>(ws, hb, lg, j0, min(kVH, nb - j0), lane);
                     __syncwarp();              // every lane is done with this half
-                    warp_stage_v<DT>(hb, tok, j0 + 2 * kVH, max(0, min(nb - j0 - 2 * kVH, kVH)), vseg, lane);
+                    warp_stage_v<DT, VQ>(hb, tok, j0 + 2 * kVH, max(0, min(nb - j0 - 2 * kVH, kVH)), vsel, lane);
                     cp_async_commit();
                 }
                 __syncwarp();                  // tok and vbuf are reused by the next batch
@@ -1112,9 +1123,9 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     }
 }
 
-template <int DT, int GM>
+template <int DT, int GM, bool VQ>
 sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStream_t stream) {
-    auto kern = decode_fused_kernel<DT, GM>;
+    auto kern = decode_fused_kernel<DT, GM, VQ>;
     const size_t smem = sizeof(FusedSmem<GM>);   // limit raised by fused_plan on this device
     FusedArgs a = args;
     void *params[] = {&a};
@@ -1128,7 +1139,7 @@ sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStr
 // concurrent first calls only repeat the same work.
 constexpr int kMaxDevices = 64;
 
-template <int DT, int GM>
+template <int DT, int GM, bool VQ>
 int occupancy_of() {
     static int cached[kMaxDevices];            // 0: unknown, else occupancy + 1
     int dev = 0;
@@ -1136,7 +1147,7 @@ int occupancy_of() {
     if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev] - 1;
     // the occupancy calculator honours the kernel's dynamic shared-memory
     // limit, which must be raised above the 48 KB default first
-    auto kern = decode_fused_kernel<DT, GM>;
+    auto kern = decode_fused_kernel<DT, GM, VQ>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FusedSmem<GM>)) !=
         cudaSuccess)
         return 0;
@@ -1172,7 +1183,7 @@ FusedLayout fused_layout(const sikv_params &p, size_t base) {
     return L;
 }
 
-FusedPlan fused_plan(const sikv_params &p) {
+FusedPlan fused_plan(const sikv_params &p, bool vq) {
     FusedPlan plan;
     const int group = p.num_q_heads / p.num_kv_heads;
     const int gm = group <= 4 ? 4 : 8;
@@ -1181,9 +1192,11 @@ FusedPlan fused_plan(const sikv_params &p) {
     if (sms <= 0) return plan;
     int occ = 0;
     if (p.dtype == SIKV_DTYPE_BF16)
-        occ = gm == 4 ? occupancy_of<SIKV_DTYPE_BF16, 4>() : occupancy_of<SIKV_DTYPE_BF16, 8>();
+        occ = vq ? (gm == 4 ? occupancy_of<SIKV_DTYPE_BF16, 4, true>() : occupancy_of<SIKV_DTYPE_BF16, 8, true>())
+                 : (gm == 4 ? occupancy_of<SIKV_DTYPE_BF16, 4, false>() : occupancy_of<SIKV_DTYPE_BF16, 8, false>());
     else
-        occ = gm == 4 ? occupancy_of<SIKV_DTYPE_F32, 4>() : occupancy_of<SIKV_DTYPE_F32, 8>();
+        occ = vq ? (gm == 4 ? occupancy_of<SIKV_DTYPE_F32, 4, true>() : occupancy_of<SIKV_DTYPE_F32, 8, true>())
+                 : (gm == 4 ? occupancy_of<SIKV_DTYPE_F32, 4, false>() : occupancy_of<SIKV_DTYPE_F32, 8, false>());
     if (occ < 1) return plan;
     int cps = (sms * occ) / segs;
     const int min_chunk = 2048;
@@ -1203,19 +1216,20 @@ FusedPlan fused_plan(const sikv_params &p) {
     return plan;
 }
 
-int fused_sub_batch(const sikv_params &p) {
+int fused_sub_batch(const sikv_params &p, bool vq) {
     // the largest number of sequences per launch whose segments fit one
     // co-resident launch (0: none does, or the whole batch already does)
     for (int bs = p.batch - 1; bs >= 1; --bs) {
         sikv_params ps = p;
         ps.batch = bs;
-        if (fused_plan(ps).ok) return bs;
+        if (fused_plan(ps, vq).ok) return bs;
     }
     return 0;
 }
 
 sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
-                                const void *V, const uint8_t *codes, const float *codebook, const float *mu,
+                                const void *V, const uint8_t *vq, const uint8_t *codes, const float *codebook,
+                                const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
                                 float *scores_out, char *ws, size_t base, int32_t *status, cudaStream_t stream) {
     const FusedLayout L = fused_layout(p, base);
@@ -1223,6 +1237,7 @@ sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, con
     a.q = q;
     a.K = K;
     a.V = V;
+    a.vq = vq;
     a.codes = codes;
     a.codebook = codebook;
     a.mu = mu;
@@ -1248,11 +1263,18 @@ sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, con
     a.part_o = reinterpret_cast<float *>(ws + L.part_o);
     a.part_ml = reinterpret_cast<float2 *>(ws + L.part_ml);
     a.status = status;
+    if (vq) {
+        if (p.dtype == SIKV_DTYPE_BF16)
+            return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_BF16, 4, true>(a, plan, stream)
+                                : launch_fused_t<SIKV_DTYPE_BF16, 8, true>(a, plan, stream);
+        return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_F32, 4, true>(a, plan, stream)
+                            : launch_fused_t<SIKV_DTYPE_F32, 8, true>(a, plan, stream);
+    }
     if (p.dtype == SIKV_DTYPE_BF16)
-        return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_BF16, 4>(a, plan, stream)
-                            : launch_fused_t<SIKV_DTYPE_BF16, 8>(a, plan, stream);
-    return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_F32, 4>(a, plan, stream)
-                        : launch_fused_t<SIKV_DTYPE_F32, 8>(a, plan, stream);
+        return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_BF16, 4, false>(a, plan, stream)
+                            : launch_fused_t<SIKV_DTYPE_BF16, 8, false>(a, plan, stream);
+    return plan.gm == 4 ? launch_fused_t<SIKV_DTYPE_F32, 4, false>(a, plan, stream)
+                        : launch_fused_t<SIKV_DTYPE_F32, 8, false>(a, plan, stream);
 }
 
 }  // namespace sikv

@@ -4,6 +4,8 @@
 // Keys" (gist.science summary of paper 2603.14224), technical summary §2.1.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -159,6 +161,24 @@ __device__ __forceinline__ float dd_div_to_float_rn(dd s, double n) {
     double ql = (r + s.lo) / n;
     dd q = fast_two_sum(qh, ql);
     return dd_to_float_rn(q.hi, q.lo);
+}
+
+// ---------------------------------------------------------------------------
+// 2-bit value rows: 32 bytes of levels (dimension d in bits 2 (d mod 4) of
+// byte d / 4), then the (min, step) fp16 pairs of the four 32-channel groups
+// ---------------------------------------------------------------------------
+
+constexpr int kVqRowBytes = 48;
+constexpr int kVqGroup = 32;
+
+// Dimensions 4 lane .. 4 lane + 3 of a quantized row: min + level * step.
+__device__ __forceinline__ float4 vq_decode4(const uint8_t *row, int lane) {
+    const uint32_t lv = row[lane];
+    const uint32_t ms = *reinterpret_cast<const uint32_t *>(row + 32 + 4 * (lane >> 3));
+    const float m = __half2float(__ushort_as_half(static_cast<unsigned short>(ms & 0xFFFFu)));
+    const float st = __half2float(__ushort_as_half(static_cast<unsigned short>(ms >> 16)));
+    return make_float4(fmaf(static_cast<float>(lv & 3u), st, m), fmaf(static_cast<float>((lv >> 2) & 3u), st, m),
+                       fmaf(static_cast<float>((lv >> 4) & 3u), st, m), fmaf(static_cast<float>(lv >> 6), st, m));
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -72,6 +72,10 @@ sikv_status launch_kmeans(const sikv_params &p, const KmeansLayout &L, const voi
                           const float *mu, const int32_t *init_idx, int iters, uint8_t *codes, float *codebook,
                           int32_t *counts, char *ws, cudaStream_t stream);
 
+// 2-bit value rows (values.cu)
+sikv_status launch_quantize_values(const sikv_params &p, const void *V, const int32_t *seq_lens, uint8_t *vq,
+                                   int32_t *status, cudaStream_t stream);
+
 sikv_status launch_append(const sikv_params &p, const void *K, const int32_t *start, const int32_t *count,
                           const float *mu, uint8_t *codes, int32_t *status, cudaStream_t stream);
 sikv_status launch_score(const sikv_params &p, const void *q, const uint8_t *codes,
@@ -83,6 +87,7 @@ sikv_status launch_topk(const sikv_params &p, const float *scores, const int32_t
                         cudaStream_t stream);
 
 sikv_status launch_sparse_attn(const sikv_params &p, const void *q, const void *K, const void *V,
+                               const uint8_t *vq,
                                const uint8_t *codes, const float *codebook, const float *mu,
                                const int32_t *idx, const int32_t *k_per_seq,
                                const int32_t *seq_lens, void *out, char *ws, size_t attn_base,
@@ -106,10 +111,12 @@ struct FusedPlan {
 };
 
 FusedLayout fused_layout(const sikv_params &p, size_t base);
-FusedPlan fused_plan(const sikv_params &p);
-int fused_sub_batch(const sikv_params &p);   // sequences per launch when the batch must be split; 0: no split
+// vq: the kernel that reads 2-bit value rows for the selected tokens
+FusedPlan fused_plan(const sikv_params &p, bool vq = false);
+int fused_sub_batch(const sikv_params &p, bool vq = false);   // sequences per launch when the batch must be split; 0: no split
 sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
-                                const void *V, const uint8_t *codes, const float *codebook, const float *mu,
+                                const void *V, const uint8_t *vq, const uint8_t *codes, const float *codebook,
+                                const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
                                 float *scores_out, char *ws, size_t base, int32_t *status, cudaStream_t stream);
 

@@ -157,3 +157,21 @@ def test_kmeans_validates_without_launch():
     assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 20, fake, fake, ctypes.c_void_p((1 << 20) + 2),
                                   fake, ws, None) == 2                                                  # misaligned counts
     assert L.sikv_kmeans_codebook(ctypes.byref(p), *args, 20, fake, fake, None, fake, 256, None) == 3   # workspace too small
+
+
+def test_value_quantization_entry_points_validate_without_launch():
+    p = _p()
+    L = sk.lib()
+    assert L.sikv_quantize_values_workspace_size(ctypes.byref(p)) == 256
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)                   # not 16-byte aligned
+    assert L.sikv_quantize_values(ctypes.byref(p), fake, fake, None, fake, 256, None) == 1
+    assert L.sikv_quantize_values(ctypes.byref(p), fake, fake, odd, fake, 256, None) == 2
+    assert L.sikv_quantize_values(ctypes.byref(p), fake, fake, fake, fake, 16, None) == 3
+    ws = L.sikv_decode_workspace_size(ctypes.byref(p))
+    args = [fake] * 9
+    assert L.sikv_decode_qv(ctypes.byref(p), fake, fake, fake, None, *args[:6], None, None, fake, ws, None) == 1
+    assert L.sikv_decode_qv(ctypes.byref(p), fake, fake, fake, odd, *args[:6], None, None, fake, ws, None) == 2
+    wa = L.sikv_sparse_attn_workspace_size(ctypes.byref(p))
+    assert L.sikv_sparse_attn_qv(ctypes.byref(p), fake, fake, fake, None, *args[:7], fake, wa, None) == 1
+    assert L.sikv_sparse_attn_qv(ctypes.byref(p), fake, fake, fake, odd, *args[:7], fake, wa, None) == 2
