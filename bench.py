@@ -65,19 +65,20 @@ def parse_args(argv=None):
 # workload arithmetic (bytes per step, the roofline numerator)
 # ----------------------------------------------------------------------------
 
-def step_bytes(w: gen.Workload) -> int:
+def step_bytes(w: gen.Workload, value_row_bytes: int | None = None) -> int:
     """Algorithmic HBM bytes of one decode step.
 
     Per (sequence, KV head): the n = N - S code rows (16 B each), the k
-    selected value rows (D x 2 B), the S sink key and value rows, and the
-    8 KB codebook.
+    selected value rows (D x 2 B, or ``value_row_bytes`` each when they are
+    read as 2-bit rows), the S sink key and value rows, and the 8 KB codebook.
     """
     eb = 4 if w.dtype == "f32" else 2
+    vrow = w.head_dim * eb if value_row_bytes is None else value_row_bytes
     tot = 0
     for b in range(w.batch):
         n = max(w.seq_lens[b] - w.num_sinks, 0)
         s = min(w.num_sinks, w.seq_lens[b])
-        per_head = 16 * n + w.topk[b] * w.head_dim * eb + s * 2 * w.head_dim * eb + 32 * 16 * 4 * 4
+        per_head = 16 * n + w.topk[b] * vrow + s * 2 * w.head_dim * eb + 32 * 16 * 4 * 4
         tot += per_head * w.num_kv_heads
     return tot
 
@@ -483,6 +484,37 @@ def run_sikv(args):
             kv_bytes / (float(measured_peaks()[0]["hbm_gbs"]) * 1e3) / (1e3 * ms_score / args.steps),
     }
 
+    # 2-bit values: the same steps with the selected tokens' values read from
+    # 48-byte 2-bit rows (sinks keep full precision); not the headline, whose
+    # values stay in the storage dtype
+    for c in reps:
+        c.quantize_values(stream=stream)
+    torch.cuda.synchronize()
+
+    def decode_qv_step(i):
+        c = reps[i % R]
+        sk.sikv_decode_qv(p, qs[i], c.K, c.V, c.vq, c.codes, c.codebook, c.mu, seq, kk, out, workspace=ws,
+                          stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            decode_qv_step(i)
+    torch.cuda.synchronize()
+    g = graph_of(decode_qv_step, args.warmup, total)
+    ms_qv = max_over_ranks(timed(g), world)
+    del g
+    ws.check()
+    sb_qv = step_bytes(w, value_row_bytes=48)
+    values_2bit = {
+        "decode_us": 1e3 * ms_qv / args.steps, "steps_per_s": world * args.steps / (ms_qv / 1e3),
+        "algorithmic_bytes_per_step": sb_qv, "GB_per_s": sb_qv / (ms_qv / 1e3 / args.steps) / 1e9,
+        "frac_of_hbm": sb_qv / (ms_qv / 1e3 / args.steps) / 1e9 / float(measured_peaks()[0]["hbm_gbs"]),
+        "value_bytes_per_selected_token": 48,
+        "note": "selected tokens' V as 2-bit rows (groups of 32 channels, fp16 min and step); sinks in bf16",
+    }
+    for c in reps:
+        c.vq = None
+
     # clustering: the one-pass sign-pattern codebook (the whole prefill
     # encoder, mean pass included) against 20 Lloyd's k-means iterations on the
     # same points (mean given), both on this GPU with this library's kernels
@@ -587,6 +619,7 @@ def run_sikv(args):
         "encode": {"ms": enc_ms, "keys_per_s": w.batch * w.num_kv_heads * w.max_seq_len / (enc_ms / 1e3),
                    "GB_per_s_2reads": 2 * K.numel() * K.element_size() / (enc_ms / 1e3) / 1e9},
         "comparison": comparison,
+        "values_2bit": values_2bit,
         "clocks": sampler.summary(),
         "gpu_launches": launches * args.steps,
         "e2e": e2e,
