@@ -24,6 +24,12 @@ def test_full_size_decode_matches_oracle_on_samples(cfg):
     dw = gu.DeviceWorkload(w)
     dw.encode()
     out, idx, sc = dw.decode()
+    # the call bench.py times (no selection or score outputs) gives the same bytes
+    bench_out = torch.empty_like(out)
+    dw.cache.decode(dw.q[0], dw.k, out=bench_out)
+    torch.cuda.synchronize()
+    assert dw.cache.ws_decode.check() == 0
+    assert torch.equal(bench_out, out)
     idx = idx.cpu().numpy()
     out = gu.to_f64(out)
     assert np.isfinite(out).all()
@@ -51,5 +57,31 @@ def test_full_size_decode_matches_oracle_on_samples(cfg):
         assert needles <= set(idx[b, h, :k].tolist())
         g = out[b, h * w.group:(h + 1) * w.group]
         assert np.allclose(g, o_out, atol=2e-2, rtol=1e-2), (cfg, b, h, float(np.abs(g - o_out).max()))
+    del dw
+    torch.cuda.empty_cache()
+
+
+def test_full_size_decode_qv_matches_oracle_on_samples():
+    """2-bit values at the long-context workload (4 x 128K), sampled segments."""
+    w = gen.config(2)
+    dw = gu.DeviceWorkload(w)
+    dw.encode()
+    dw.cache.quantize_values()
+    out = torch.empty((w.batch, w.num_q_heads, 128), dtype=dw.p.torch_dtype, device=dw.dev)
+    dw.cache.decode_qv(dw.q[0], dw.k, out=out)
+    torch.cuda.synchronize()
+    assert dw.cache.ws_decode.check() == 0 and dw.cache.ws_encode.check() == 0
+    out = gu.to_f64(out)
+    assert np.isfinite(out).all()
+    for (b, h) in SAMPLES[2]:
+        k = w.topk[b]
+        o = gu.oracle_head(w, dw.bt, b, h)
+        q = gu.oracle_queries(w, dw.bt, 0, b, h)
+        vq = dw.cache.vq[b, h, :w.seq_lens[b]].cpu().numpy()
+        packed = oracle.quantize_values(o.V)
+        assert np.array_equal(vq, packed)
+        o_out, _, _, _ = oracle.decode_step_qv(q, o.K, o.V, packed, o.mu, o.cent, o.code, k, w.num_sinks)
+        g = out[b, h * w.group:(h + 1) * w.group]
+        assert np.allclose(g, o_out, atol=2e-2, rtol=1e-2), (b, h, float(np.abs(g - o_out).max()))
     del dw
     torch.cuda.empty_cache()
