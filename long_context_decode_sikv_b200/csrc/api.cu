@@ -135,13 +135,20 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
     const bool qv = vq != nullptr;
     const FusedPlan plan = fused_plan(*p, qv);
     if (plan.ok)
-        return launch_decode_fused(*p, plan, q, K, V, vq, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
-                                   scores_out, ws, L.fused, status, s);
+        return launch_decode_fused(*p, plan, fused_layout(*p, L.fused), q, K, V, vq, codes, codebook, mu, seq_lens,
+                                   k_per_seq, out, idx_out, scores_out, ws, status, s);
     // Too many segments for one co-resident launch: run the single-launch
     // kernel on sub-batches of sequences that fit, one after the other on the
     // stream (each launch leaves the coordination state zeroed for the next).
     const int bsub = fused_sub_batch(*p, qv);
     if (bsub > 0) {
+        // one coordination layout, the largest sub-batch's, for every
+        // sub-launch: a layout sized by each launch's own batch would place
+        // one launch's counters and candidates over another's histograms,
+        // which no launch then clears
+        sikv_params pmax = *p;
+        pmax.batch = bsub;
+        const FusedLayout FL = fused_layout(pmax, L.fused);
         const size_t eb = p->dtype == SIKV_DTYPE_F32 ? 4 : 2;
         const size_t hq = p->num_q_heads, hkv = p->num_kv_heads, nmax = p->max_seq_len, d = p->head_dim;
         for (int b0 = 0; b0 < p->batch; b0 += bsub) {
@@ -151,14 +158,14 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
             if (!pl.ok) return SIKV_ERR_UNSUPPORTED;      // cannot happen: fused_sub_batch checked it
             const size_t bq = static_cast<size_t>(b0) * hq * d * eb, bkv = static_cast<size_t>(b0) * hkv * nmax * d * eb;
             SIKV_TRY(launch_decode_fused(
-                ps, pl, static_cast<const char *>(q) + bq, static_cast<const char *>(K) + bkv,
+                ps, pl, FL, static_cast<const char *>(q) + bq, static_cast<const char *>(K) + bkv,
                 static_cast<const char *>(V) + bkv,
                 qv ? vq + static_cast<size_t>(b0) * hkv * nmax * kVqRowBytes : nullptr,
                 codes + static_cast<size_t>(b0) * hkv * nmax * (d / 8),
                 codebook + static_cast<size_t>(b0) * hkv * kSubspaces * kClusters * 4,
                 mu + static_cast<size_t>(b0) * hkv * d, seq_lens + b0, k_per_seq + b0, static_cast<char *>(out) + bq,
                 idx_out ? idx_out + static_cast<size_t>(b0) * hkv * (p->max_topk > 0 ? p->max_topk : 0) : nullptr,
-                scores_out ? scores_out + static_cast<size_t>(b0) * hkv * nmax : nullptr, ws, L.fused, status, s));
+                scores_out ? scores_out + static_cast<size_t>(b0) * hkv * nmax : nullptr, ws, status, s));
         }
         return SIKV_OK;
     }

@@ -1227,12 +1227,11 @@ int fused_sub_batch(const sikv_params &p, bool vq) {
     return 0;
 }
 
-sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
-                                const void *V, const uint8_t *vq, const uint8_t *codes, const float *codebook,
-                                const float *mu,
+sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const FusedLayout &L, const void *q,
+                                const void *K, const void *V, const uint8_t *vq, const uint8_t *codes,
+                                const float *codebook, const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
-                                float *scores_out, char *ws, size_t base, int32_t *status, cudaStream_t stream) {
-    const FusedLayout L = fused_layout(p, base);
+                                float *scores_out, char *ws, int32_t *status, cudaStream_t stream) {
     FusedArgs a;
     a.q = q;
     a.K = K;

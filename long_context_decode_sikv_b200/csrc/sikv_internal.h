@@ -114,11 +114,13 @@ FusedLayout fused_layout(const sikv_params &p, size_t base);
 // vq: the kernel that reads 2-bit value rows for the selected tokens
 FusedPlan fused_plan(const sikv_params &p, bool vq = false);
 int fused_sub_batch(const sikv_params &p, bool vq = false);   // sequences per launch when the batch must be split; 0: no split
-sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const void *q, const void *K,
-                                const void *V, const uint8_t *vq, const uint8_t *codes, const float *codebook,
-                                const float *mu,
+// L: the coordination layout in ws; every launch that shares ws must use the
+// same layout, because each launch leaves only its own segments' state zeroed
+sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, const FusedLayout &L, const void *q,
+                                const void *K, const void *V, const uint8_t *vq, const uint8_t *codes,
+                                const float *codebook, const float *mu,
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
-                                float *scores_out, char *ws, size_t base, int32_t *status, cudaStream_t stream);
+                                float *scores_out, char *ws, int32_t *status, cudaStream_t stream);
 
 int device_sm_count();
 
