@@ -16,13 +16,17 @@
 // The codes are the last assignment, packed like the sign codes (two per
 // byte, even subspace in the low nibble), so the LUT scorer reads them as is.
 //
-// One launch of kmeans_iter_kernel per iteration, then kmeans_update_kernel:
-//   iter    lane l of a warp owns subspace l: the warp reads one key row per
+// Per iteration: kmeans_assign_kernel, kmeans_accum_kernel, kmeans_update_kernel.
+//   assign  lane l of a warp owns subspace l: the warp reads one key row per
 //           token (coalesced), each lane finds its sub-vector's nearest of 16
 //           centroids held in registers (differences and squares of two
-//           clusters per f32x2 instruction, then a tree argmin), and adds the point exactly
-//           (double-double) to its warp's shared-memory sums.  The CTA merges
-//           its warps in a fixed order and writes one partial per chunk.
+//           clusters per f32x2 instruction, then a tree argmin) and the 8
+//           lanes of each 32-bit word store the packed codes.
+//   accum   thread d owns channel d: for each token of its chunk it adds
+//           fl32(k_d - mu_d) exactly (double-double) to the sum of the token's
+//           cluster in its own shared-memory column (16 clusters x 16 bytes),
+//           so accesses never conflict and many CTAs share an SM; one partial
+//           per chunk.
 //   update  per (segment, subspace, cluster, dim): the chunk partials in chunk
 //           order, then the correctly rounded quotient by the count.
 // The sums are exact while a cluster's points span fewer than about 40
@@ -34,21 +38,23 @@ namespace sikv {
 
 namespace {
 
-constexpr int kKmWarps = 4;                    // one warp per SM sub-partition
+constexpr int kKmWarps = 4;                    // assign: 4 warps per CTA, several CTAs per SM
 constexpr int kKmThreads = kKmWarps * 32;
-constexpr int kKmUnroll = 8;                   // key rows per group; two groups in flight per warp
+constexpr int kKmUnroll = 4;                   // key rows per group; two groups in flight per warp
 constexpr int kKmClusters = 16;
 constexpr int kKmSub = kHeadDim / 4;           // 32 subspaces: one per lane
 constexpr int kKmEntries = kKmClusters * 4 * kKmSub;   // (cluster, dim, subspace) sums
 constexpr int kKmUpdateThreads = 256;
+constexpr int kKaThreads = kHeadDim;           // accum: one thread per channel
+constexpr int kKaUnroll = 8;                   // keys loaded ahead per thread
+constexpr int kKmCtasPerSm = 6;                // accum CTAs per SM the chunking aims for
 
-// One warp's exact sums, [cluster][dim][subspace]: lane l touches column l
-// only, so a warp's 16-byte accesses are conflict-free whatever the clusters.
-struct KmWarpAcc {
-    double2 sum[kKmClusters][4][kKmSub];       // (hi, lo) double-double, 32 KB
-    int32_t cnt[kKmClusters][kKmSub];          // 2 KB
+// One accumulation CTA's exact sums: column d (channel d) belongs to thread
+// d, so a warp's 16-byte accesses are conflict-free whatever the clusters.
+struct KmAccSmem {
+    double2 sum[kKmClusters][kKaThreads];      // (hi, lo) double-double, 32 KB
+    int32_t cnt[kKmClusters][kKmSub];          // 2 KB (threads of dimension 0 count)
 };
-constexpr size_t kKmSmem = sizeof(KmWarpAcc) * kKmWarps;
 
 __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
     return static_cast<unsigned long long>(__float_as_uint(lo)) |
@@ -112,19 +118,6 @@ __device__ __forceinline__ dd dd_merge(dd a, dd b) {
     return two_sum(r.hi, r.lo);
 }
 
-__device__ __forceinline__ void acc_point(KmWarpAcc &A, int a, int lane, float x0, float x1, float x2, float x3) {
-    const float xs[4] = {x0, x1, x2, x3};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        double2 v = A.sum[a][i][lane];
-        const dd t = two_sum(v.x, static_cast<double>(xs[i]));
-        v.x = t.hi;
-        v.y += t.lo;
-        A.sum[a][i][lane] = v;
-    }
-    A.cnt[a][lane] += 1;
-}
-
 // Starting centroids: c[s][j][i] = fl32(K[init_j][4s+i] - mu[4s+i]).  A
 // segment with no non-sink token, an invalid length or an invalid start
 // token gets 0 for the affected centroids (the latter two flagged).
@@ -155,31 +148,20 @@ kmeans_init_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_l
     }
 }
 
-// One assignment pass over chunk blockIdx.x of segment blockIdx.y: exact
-// per-cluster sums and counts into part_sum / part_cnt, and (last iteration
-// only, codes != nullptr) the packed assignment of every token.
+// Assignment of the tokens of chunk blockIdx.x of segment blockIdx.y: the
+// packed nearest-centroid codes of every token into codes.
 template <int DT>
-__global__ void __launch_bounds__(kKmThreads, 1)
-kmeans_iter_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_lens, const float *__restrict__ mu,
-                   const float *__restrict__ cent, int hkv, int nmax, int num_sinks, int chunk, int nchunks,
-                   double2 *__restrict__ part_sum, int32_t *__restrict__ part_cnt, uint8_t *__restrict__ codes,
-                   int32_t *status) {
+__global__ void __launch_bounds__(kKmThreads)
+kmeans_assign_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_lens, const float *__restrict__ mu,
+                     const float *__restrict__ cent, int hkv, int nmax, int num_sinks, int chunk,
+                     uint8_t *__restrict__ codes, int32_t *status) {
     constexpr int EB = ElemBytes<DT>::value;
-    extern __shared__ __align__(16) unsigned char km_smem[];
-    KmWarpAcc *acc = reinterpret_cast<KmWarpAcc *>(km_smem);
     const int seg = blockIdx.y, c = blockIdx.x;
     const int n_tok = load_seq_len(seq_lens, seg / hkv, nmax, status);
     const int t0 = num_sinks + c * chunk;
-    if (n_tok < 0 || t0 >= n_tok) return;                                 // block-uniform
+    if (n_tok < 0 || t0 >= n_tok) return;
     const int t1 = min(n_tok, t0 + chunk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    for (int w = 0; w < kKmWarps; ++w) {
-        double2 *sums = &acc[w].sum[0][0][0];
-        int32_t *cnts = &acc[w].cnt[0][0];
-        for (int e = threadIdx.x; e < kKmEntries; e += kKmThreads) sums[e] = make_double2(0.0, 0.0);
-        for (int e = threadIdx.x; e < kKmClusters * kKmSub; e += kKmThreads) cnts[e] = 0;
-    }
 
     // this lane's subspace: its 16 centroids (as pairs) and 4 mean entries
     unsigned long long cp[kKmClusters / 2][4];
@@ -193,11 +175,9 @@ kmeans_iter_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_l
         cp[p][3] = pack2(a.w, b.w);
     }
     const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mu + static_cast<size_t>(seg) * kHeadDim) + lane);
-    __syncthreads();
-
-    KmWarpAcc &A = acc[warp];
     const char *krows = static_cast<const char *>(K) + static_cast<size_t>(seg) * nmax * kHeadDim * EB;
-    uint32_t *crow = codes ? reinterpret_cast<uint32_t *>(codes) + static_cast<size_t>(seg) * nmax * 4 : nullptr;
+    uint32_t *crow = reinterpret_cast<uint32_t *>(codes) + static_cast<size_t>(seg) * nmax * 4;
+
     // rows t, t + W, ..., t + (U-1) W of this warp; the next group is loaded
     // before the current one is processed, so its latency overlaps the work
     float4 cur[kKmUnroll];
@@ -218,42 +198,82 @@ kmeans_iter_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_l
         for (int u = 0; u < kKmUnroll; ++u) {
             const int tu = t + u * kKmWarps;
             if (tu < t1) {                              // warp-uniform
-                const float x0 = __fsub_rn(cur[u].x, m4.x), x1 = __fsub_rn(cur[u].y, m4.y);
-                const float x2 = __fsub_rn(cur[u].z, m4.z), x3 = __fsub_rn(cur[u].w, m4.w);
-                const int a = nearest(cp, x0, x1, x2, x3);
-                acc_point(A, a, lane, x0, x1, x2, x3);
-                if (crow) {
-                    uint32_t word = static_cast<uint32_t>(a) << (4 * (lane & 7));
+                const int a = nearest(cp, __fsub_rn(cur[u].x, m4.x), __fsub_rn(cur[u].y, m4.y),
+                                      __fsub_rn(cur[u].z, m4.z), __fsub_rn(cur[u].w, m4.w));
+                uint32_t word = static_cast<uint32_t>(a) << (4 * (lane & 7));
 #pragma unroll
-                    for (int off = 1; off < 8; off <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, off);
-                    if ((lane & 7) == 0) crow[static_cast<size_t>(tu) * 4 + (lane >> 3)] = word;
-                }
+                for (int off = 1; off < 8; off <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, off);
+                if ((lane & 7) == 0) crow[static_cast<size_t>(tu) * 4 + (lane >> 3)] = word;
             }
         }
 #pragma unroll
         for (int u = 0; u < kKmUnroll; ++u) cur[u] = nxt[u];
         t = tn;
     }
-    __syncthreads();
+}
 
-    // the warps' sums in warp order -> this chunk's partial
+// Exact per-cluster sums and counts of chunk blockIdx.x of segment
+// blockIdx.y under the codes of this iteration, into part_sum / part_cnt
+// (entry (cluster, dim, subspace) = (a * 4 + i) * 32 + s).
+template <int DT>
+__global__ void __launch_bounds__(kKaThreads)
+kmeans_accum_kernel(const void *__restrict__ K, const int32_t *__restrict__ seq_lens, const float *__restrict__ mu,
+                    const uint8_t *__restrict__ codes, int hkv, int nmax, int num_sinks, int chunk, int nchunks,
+                    double2 *__restrict__ part_sum, int32_t *__restrict__ part_cnt, int32_t *status) {
+    constexpr int EB = ElemBytes<DT>::value;
+    extern __shared__ __align__(16) unsigned char km_smem[];
+    KmAccSmem &A = *reinterpret_cast<KmAccSmem *>(km_smem);
+    const int seg = blockIdx.y, c = blockIdx.x;
+    const int n_tok = load_seq_len(seq_lens, seg / hkv, nmax, status);
+    const int t0 = num_sinks + c * chunk;
+    if (n_tok < 0 || t0 >= n_tok) return;               // block-uniform
+    const int t1 = min(n_tok, t0 + chunk);
+    const int d = threadIdx.x, s = d >> 2, i = d & 3;
+#pragma unroll
+    for (int a = 0; a < kKmClusters; ++a) A.sum[a][d] = make_double2(0.0, 0.0);
+    if (i == 0) {
+#pragma unroll
+        for (int a = 0; a < kKmClusters; ++a) A.cnt[a][s] = 0;
+    }
+    const float m = __ldg(mu + static_cast<size_t>(seg) * kHeadDim + d);
+    const char *krows = static_cast<const char *>(K) + static_cast<size_t>(seg) * nmax * kHeadDim * EB;
+    const uint8_t *cbytes = codes + static_cast<size_t>(seg) * nmax * kCodeBytes + (s >> 1);
+    const int shift = 4 * (s & 1);
+#pragma unroll 1
+    for (int t = t0; t < t1; t += kKaUnroll) {
+        float v[kKaUnroll];
+        uint32_t cb[kKaUnroll];
+#pragma unroll
+        for (int u = 0; u < kKaUnroll; ++u) {
+            const bool ok = t + u < t1;
+            v[u] = ok ? load1<DT>(krows + static_cast<size_t>(t + u) * kHeadDim * EB, d) : 0.f;
+            cb[u] = ok ? __ldg(cbytes + static_cast<size_t>(t + u) * kCodeBytes) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kKaUnroll; ++u) {
+            if (t + u >= t1) break;
+            const int a = static_cast<int>((cb[u] >> shift) & 15u);
+            double2 acc = A.sum[a][d];
+            const dd r = two_sum(acc.x, static_cast<double>(__fsub_rn(v[u], m)));
+            acc.x = r.hi;
+            acc.y += r.lo;
+            A.sum[a][d] = acc;
+            if (i == 0) A.cnt[a][s] += 1;
+        }
+    }
+    // this thread's sums (its own column) and counts -> the chunk's partial
     const size_t pbase = static_cast<size_t>(seg) * nchunks + c;
     double2 *ps = part_sum + pbase * kKmEntries;
-    for (int e = threadIdx.x; e < kKmEntries; e += kKmThreads) {
-        dd s = {0.0, 0.0};
 #pragma unroll
-        for (int w = 0; w < kKmWarps; ++w) {
-            const double2 v = (&acc[w].sum[0][0][0])[e];
-            s = dd_merge(s, dd{v.x, v.y});
-        }
-        ps[e] = make_double2(s.hi, s.lo);
+    for (int a = 0; a < kKmClusters; ++a) {
+        const double2 acc = A.sum[a][d];
+        const dd r = two_sum(acc.x, acc.y);
+        ps[(a * 4 + i) * kKmSub + s] = make_double2(r.hi, r.lo);
     }
-    int32_t *pc = part_cnt + pbase * kKmClusters * kKmSub;
-    for (int e = threadIdx.x; e < kKmClusters * kKmSub; e += kKmThreads) {
-        int n = 0;
+    if (i == 0) {
+        int32_t *pc = part_cnt + pbase * kKmClusters * kKmSub;
 #pragma unroll
-        for (int w = 0; w < kKmWarps; ++w) n += acc[w].cnt[e / kKmSub][e % kKmSub];
-        pc[e] = n;
+        for (int a = 0; a < kKmClusters; ++a) pc[a * kKmSub + s] = A.cnt[a][s];
     }
 }
 
@@ -291,8 +311,8 @@ KmeansLayout kmeans_layout(const sikv_params &p, int num_sms) {
     KmeansLayout L;
     const int segs = p.batch * p.num_kv_heads;
     const int pts = std::max(p.max_seq_len - p.num_sinks, 1);
-    // one wave: as many chunks per segment as the SMs allow (one CTA per SM)
-    const int per_seg = std::max(1, std::min(num_sms / segs, (pts + 255) / 256));
+    // about kKmCtasPerSm accumulation CTAs per SM, chunks of at least 256 tokens
+    const int per_seg = std::max(1, std::min(kKmCtasPerSm * num_sms / segs, (pts + 255) / 256));
     L.chunk = (pts + per_seg - 1) / per_seg;
     L.nchunks = (pts + L.chunk - 1) / L.chunk;
     size_t off = kHeaderBytes;
@@ -312,9 +332,10 @@ sikv_status launch_kmeans(const sikv_params &p, const KmeansLayout &L, const voi
     double2 *psum = reinterpret_cast<double2 *>(ws + L.part_sum);
     int32_t *pcnt = reinterpret_cast<int32_t *>(ws + L.part_cnt);
     const bool bf16 = p.dtype == SIKV_DTYPE_BF16;
-    auto iter = bf16 ? kmeans_iter_kernel<SIKV_DTYPE_BF16> : kmeans_iter_kernel<SIKV_DTYPE_F32>;
-    if (cudaFuncSetAttribute(iter, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kKmSmem)) !=
-        cudaSuccess)
+    auto accum = bf16 ? kmeans_accum_kernel<SIKV_DTYPE_BF16> : kmeans_accum_kernel<SIKV_DTYPE_F32>;
+    auto assign = bf16 ? kmeans_assign_kernel<SIKV_DTYPE_BF16> : kmeans_assign_kernel<SIKV_DTYPE_F32>;
+    const size_t smem = sizeof(KmAccSmem);
+    if (cudaFuncSetAttribute(accum, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return SIKV_ERR_CUDA;
     if (bf16)
         kmeans_init_kernel<SIKV_DTYPE_BF16><<<segs, 256, 0, stream>>>(K, seq_lens, mu, init_idx, codebook,
@@ -324,11 +345,13 @@ sikv_status launch_kmeans(const sikv_params &p, const KmeansLayout &L, const voi
         kmeans_init_kernel<SIKV_DTYPE_F32><<<segs, 256, 0, stream>>>(K, seq_lens, mu, init_idx, codebook,
                                                                      p.num_kv_heads, p.max_seq_len, p.num_sinks,
                                                                      status);
+    const dim3 grid(L.nchunks, segs);
     for (int it = 0; it < iters; ++it) {
         const bool last = it == iters - 1;
-        iter<<<dim3(L.nchunks, segs), kKmThreads, kKmSmem, stream>>>(K, seq_lens, mu, codebook, p.num_kv_heads,
-                                                                    p.max_seq_len, p.num_sinks, L.chunk, L.nchunks,
-                                                                    psum, pcnt, last ? codes : nullptr, status);
+        assign<<<grid, kKmThreads, 0, stream>>>(K, seq_lens, mu, codebook, p.num_kv_heads, p.max_seq_len,
+                                                p.num_sinks, L.chunk, codes, status);
+        accum<<<grid, kKaThreads, smem, stream>>>(K, seq_lens, mu, codes, p.num_kv_heads, p.max_seq_len, p.num_sinks,
+                                                  L.chunk, L.nchunks, psum, pcnt, status);
         kmeans_update_kernel<<<segs, kKmUpdateThreads, 0, stream>>>(seq_lens, p.num_kv_heads, p.max_seq_len,
                                                                    p.num_sinks, L.chunk, L.nchunks, psum, pcnt,
                                                                    codebook, last ? counts : nullptr, status);
