@@ -19,7 +19,11 @@
  * Conventions shared by every entry point
  * ----------------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
- *    never allocates device memory and keeps no global mutable state.  Every
+ *    never allocates device memory.  Its only global state is (a) per-device
+ *    launch facts computed on the first call on each device (a kernel's
+ *    shared-memory limit, its occupancy and cluster occupancy, each written
+ *    once with the same value by any thread) and (b) the fixed scratch array
+ *    of sikv_sparse_attn_static with its per-device address cache.  Every
  *    call only enqueues kernels on `stream` and returns without synchronizing.
  *  - Scratch memory comes from the caller's `workspace` (device, 256-byte
  *    aligned, at least sikv_*_workspace_size() bytes).  Zero the whole
@@ -359,8 +363,11 @@ SIKV_API sikv_status sikv_kmeans_codebook(const sikv_params *p, const void *K, c
  *    plus 256, must fit in 8 MiB; larger sizes return SIKV_ERR_WORKSPACE and
  *    launch nothing.  Invalid parameters return SIKV_ERR_INVALID_ARG.
  *  - The first call on each device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    that device current) and caches it for the life of the process; make
+ *    that first call before any stream capture.  The cache does not survive
+ *    cudaDeviceReset (or any teardown of the device's primary context): after
+ *    one, the cached address is stale and this entry point must not be called
+ *    again in that process.
  *  - All calls share the one array: calls that may overlap on the GPU (on
  *    different streams, or from different threads) race and must be ordered
  *    by the caller.

@@ -1,6 +1,7 @@
 // Public C ABI of libsikv: argument validation, workspace sizing and the
 // entry points declared in sikv.h.
 #include <math.h>
+#include <atomic>
 #include <string.h>
 
 #include "sikv_common.cuh"
@@ -77,12 +78,16 @@ DecodeLayout decode_layout(const sikv_params &p) {
 }
 
 int device_sm_count() {
-    static int cached[64];                     // per device, 0 until first asked
+    // per device, 0 until first asked; concurrent first calls store the same value
+    static std::atomic<int> cached[64];
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    if (dev >= 0 && dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) cached[dev] = n;
+    if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 

@@ -32,28 +32,16 @@
 // Code size matters here: every phase but the scoring loop runs once per CTA
 // with a cold instruction cache, so loops over a thread's tokens stay rolled
 // (their state lives in shared memory, not in registers).
-#include "score_device.cuh"
+#include <atomic>
+
+#include "decode_common.cuh"
 #include "sikv_internal.h"
 
 namespace sikv {
 
 namespace {
 
-constexpr int kFT = 256;                 // threads per CTA
-constexpr int kFW = kFT / 32;            // warps per CTA
-constexpr int kFBins = 1024;             // histogram bins per segment
-constexpr int kFListCap = 2048;          // attended tokens staged per window
-constexpr int kFMaxNpt = 64;             // token slots per thread at most
-constexpr int kFMaxChunk = kFMaxNpt * kFT;
-constexpr int kFRankMax = 512;           // up to this many candidates: rank directly
-constexpr int kFUnroll = 4;              // code rows in flight per thread
-constexpr int kFPrefetchRows = 16;       // code rows per thread sent to L2 during the prologue
-constexpr int kFPend = kFBins / 4;       // threshold-bin tokens of a CTA re-scored together
-constexpr int kFDirect = kFBins / 2;     // attended tokens listed directly during the scans
-constexpr int kFWarpList = kFDirect / kFW;   // of which each warp lists (and attends) at most this many
-constexpr int kFVBytes = 4096;           // value rows staged per warp: 16 bf16 or 8 fp32 rows
 constexpr int kSpinLimit = 1 << 23;      // polls of a wait: seconds, far above any real wait
-constexpr int kFRow = 256;               // tokens per row scan of a warp (32 lanes x 8)
 
 struct FusedArgs {
     const void *q, *K, *V;
@@ -126,10 +114,6 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
     return v;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // Thread 0 waits until *ctr >= target (bounded); the CTA then synchronizes.
 // The acquire load orders every later read of the CTA after the arrivals.
 __device__ __forceinline__ void cta_wait(const int *ctr, int target, int32_t *status) {
@@ -159,300 +143,6 @@ __device__ __forceinline__ int cta_arrive(int *ctr) {
     return old;
 }
 
-// Exclusive scan over the CTA (256 threads) of one value per thread.
-__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t *wtot, uint32_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    if (lane == 31) wtot[warp] = incl;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t run = 0;
-        for (int w = 0; w < kFW; ++w) {
-            const uint32_t t = wtot[w];
-            wtot[w] = run;
-            run += t;
-        }
-        wtot[kFW] = run;
-    }
-    __syncthreads();
-    const uint32_t r = wtot[warp] + incl - v;
-    *total = wtot[kFW];
-    __syncthreads();
-    return r;
-}
-
-// In a histogram of PER * 256 bins scanned from the top bin down, finds the
-// bin where the running count first reaches `need` (1 <= need <= total).
-// Each thread loads its PER consecutive bins once.  Writes (bin, count above)
-// to out[0..1]; out is left untouched when the total is below need.  Ends
-// synchronized.
-template <int PER, typename Load>
-__device__ __forceinline__ void cta_find_bin(Load load, uint32_t need, uint32_t *wtot, uint32_t *out) {
-    const int top = PER * kFT - 1 - static_cast<int>(threadIdx.x) * PER;
-    uint32_t h[PER];
-    uint32_t loc = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        h[i] = load(top - i);
-        loc += h[i];
-    }
-    uint32_t total;
-    uint32_t above = cta_excl_scan(loc, wtot, &total);
-    if (above < need && need <= above + loc) {
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            if (above < need && above + h[i] >= need) {
-                out[0] = static_cast<uint32_t>(top - i);
-                out[1] = above;
-            }
-            above += h[i];
-        }
-    }
-    __syncthreads();
-}
-
-// Radix select over `n` elements (element e has key key(e) and passes
-// keep(e)): returns the key of rank `need` counted from the largest and, in
-// *need_left, how many elements equal to it are still needed.  Uses hist[0..255].
-template <typename KeyF, typename KeepF>
-__device__ __noinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, uint32_t need, uint32_t *hist,
-                                                  uint32_t *wtot, uint32_t *sc, uint32_t *need_left) {
-    uint32_t prefix = 0, mask = 0;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += kFT) hist[i] = 0;
-        __syncthreads();
-        for (int e = threadIdx.x; e < n; e += kFT) {
-            if (!keep(e)) continue;
-            const uint32_t k = key(e);
-            if (((k ^ prefix) & mask) == 0) atomicAdd(&hist[(k >> shift) & 255u], 1u);
-        }
-        __syncthreads();
-        cta_find_bin<1>([&](int i) { return hist[i]; }, need, wtot, sc);
-        prefix |= sc[0] << shift;
-        mask |= 255u << shift;
-        need -= sc[1];
-        __syncthreads();
-    }
-    *need_left = need;
-    return prefix;
-}
-
-// bins[] holds one 16-bit entry per token of the chunk in token order (entry
-// p is token t0 + p).  A lane scans 8 consecutive entries with one 16-byte
-// load; these give, per 16-bit half of each word, an all-ones mask where the
-// entry's bin is above / equal to a threshold (entries hold bin + 1).
-__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return __vcmpgtu2(w & 0x3FFF3FFFu, thr2); }
-__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) { return __vcmpeq2(w & 0x3FFF3FFFu, thr2); }
-// 8-bit mask (bit j = entry j of the lane's 8) from four per-half masks
-__device__ __forceinline__ uint32_t mask8(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
-    return (m0 & 1u) | ((m0 >> 15) & 2u) | ((m1 & 1u) << 2) | ((m1 >> 13) & 8u) | ((m2 & 1u) << 4) |
-           ((m2 >> 11) & 32u) | ((m3 & 1u) << 6) | ((m3 >> 9) & 128u);
-}
-
-// Appends the tokens of bin b* (entries equal to b2 in both halves) to the
-// segment's candidate list one by one with their exact keys, each re-scored
-// by the lane that scored it (same table, same rotation, same order of
-// additions, so bit-identical).  The fallback for a CTA whose threshold bin
-// holds more tokens than the shared list takes; ties-heavy tables only.
-__device__ __noinline__ void emit_bin_tokens(const uint16_t *bins, int nrows, uint32_t b2, const float *t2,
-                                             const uint4 *crow, int t0, float qmu, int *ncand, uint2 *cand, int cap) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
-        const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
-        // token t0 + p was scored by lane p mod 32 (the table's bank rotation)
-        uint32_t todo = __ballot_sync(0xffffffffu, eq != 0);
-        while (todo) {
-            const int src = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const uint32_t em = __shfl_sync(0xffffffffu, eq, src);
-            for (uint32_t mm = em; mm; mm &= mm - 1) {
-                const int p = row * kFRow + 8 * src + __ffs(mm) - 1;
-                if (lane == (p & 31)) {
-                    const float sv = lut2_score(t2, __ldg(crow + t0 + p), lane, qmu);
-                    const int slot = atomicAdd(ncand, 1);
-                    if (slot < cap) cand[slot] = make_uint2(score_key(sv), static_cast<uint32_t>(t0 + p));
-                }
-            }
-        }
-    }
-}
-
-// Turns sh.rowcnt-style per-row counts into exclusive prefix sums in place and
-// returns the total.  Expects the counts to be visible; ends synchronized.
-__device__ __forceinline__ uint32_t rows_to_bases(uint32_t *rowcnt, int nrows, uint32_t *wtot) {
-    uint32_t total;
-    const int tid = threadIdx.x;
-    const uint32_t v = tid < nrows ? rowcnt[tid] : 0u;
-    const uint32_t run = cta_excl_scan(v, wtot, &total);
-    if (tid < nrows) rowcnt[tid] = run;
-    __syncthreads();
-    return total;
-}
-
-// 8-bit mask of the entries of row `row` (8 per lane) that carry flag bit2.
-__device__ __forceinline__ uint32_t flagged8(const uint16_t *bins, int row, int lane, uint32_t bit2) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
-    return mask8(__vcmpne2(w.x & bit2, 0u), __vcmpne2(w.y & bit2, 0u), __vcmpne2(w.z & bit2, 0u),
-                 __vcmpne2(w.w & bit2, 0u));
-}
-
-// Fills list[0, wn) with the tokens of the entries flagged bit2 whose
-// ordinals (ascending token order) lie in [wbase, wbase + wn).  The fallback
-// when a pass holds more tokens than the direct list takes.  Ends synchronized.
-// (Inlined: as a call it costs the kernel spills around the call site.)
-__device__ __forceinline__ void stage_flagged(const uint16_t *bins, int nrows, uint32_t bit2, uint32_t wbase, int t0,
-                                           uint32_t *rowcnt, uint32_t *wtot, int32_t *list) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
-        uint32_t cnt = __popc(flagged8(bins, row, lane, bit2));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-        if (lane == 0) rowcnt[row] = cnt;
-    }
-    __syncthreads();
-    rows_to_bases(rowcnt, nrows, wtot);
-#pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
-        const uint32_t m = flagged8(bins, row, lane, bit2);
-        uint32_t incl = __popc(m);
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t o2 = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o2;
-        }
-        uint32_t ord = rowcnt[row] + incl - __popc(m);
-        for (uint32_t mm = m; mm; mm &= mm - 1, ++ord) {
-            const int t = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
-            if (ord >= wbase && ord < wbase + kFListCap) list[ord - wbase] = t;
-        }
-    }
-    __syncthreads();
-}
-
-// Online-softmax state of one warp: running max m and sum l per head (equal
-// in every lane) and the lane's four output columns (4 lane .. 4 lane + 3).
-template <int GM>
-struct WarpSoftmax {
-    float m[GM], l[GM], o[GM][4];
-};
-
-// A batch of up to 32 entries, one per lane (logit -INFINITY: no entry).
-// Folds the batch's maximum into m, rescales l and o, adds the batch's
-// weights to l and turns lg into the lane's weight exp(lg - m).
-template <int GM>
-__device__ __forceinline__ void warp_softmax_batch(WarpSoftmax<GM> &s, float (&lg)[GM]) {
-#pragma unroll
-    for (int g = 0; g < GM; ++g) {
-        float mx = lg[g];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float mn = fmaxf(s.m[g], mx);
-        const float alpha = (s.m[g] == -INFINITY) ? 0.f : __expf(s.m[g] - mn);
-        const float pr = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - mn);
-        float sum = pr;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        s.l[g] = fmaf(s.l[g], alpha, sum);
-        s.m[g] = mn;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) s.o[g][i] *= alpha;
-        lg[g] = pr;
-    }
-}
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-
-// Closes the current group of this thread's cp.async copies.
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-// Waits until at most one group of this thread's copies is still in flight.
-__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
-// Value rows staged by a warp: two halves of its buffer, so that one half
-// is consumed while the other is in flight.
-template <int DT, bool VQ>
-struct VStage {
-    static constexpr int kRowBytes = VQ ? kVqRowBytes : kHeadDim * ElemBytes<DT>::value;
-    static constexpr int kHalf = VQ ? 16 : kFVBytes / kRowBytes / 2;  // 16 (2-bit), 8 (bf16) or 4 (fp32) rows
-};
-
-// Starts copying the value rows of tokens tok[j0 .. j0 + n) into vb (row j
-// at j * kRowBytes), 16 bytes per copy, all in flight at once.
-template <int DT, bool VQ>
-__device__ __forceinline__ void warp_stage_v(char *vb, const int32_t *tok, int j0, int n, const char *vseg,
-                                             int lane) {
-    constexpr int kRowBytes = VStage<DT, VQ>::kRowBytes, kChunks = kRowBytes / 16;
-#pragma unroll 1
-    for (int i = lane; i < n * kChunks; i += 32) {
-        const int j = i / kChunks, cc = i % kChunks;
-        cp_async16(vb + j * kRowBytes + 16 * cc,
-                   vseg + static_cast<size_t>(tok[j0 + j]) * kRowBytes + 16 * cc);
-    }
-}
-
-// o += sum over the staged rows j < n of pr_{j0+j} V[row j]; lane l takes
-// columns 4l..4l+3 (a 2-bit row is read back as min + level * step).
-template <int DT, int GM, bool VQ>
-__device__ __forceinline__ void warp_fma_v(WarpSoftmax<GM> &s, const char *vb, const float (&pr)[GM], int j0, int n,
-                                           int lane) {
-    constexpr int kRowBytes = VStage<DT, VQ>::kRowBytes;
-#pragma unroll 2
-    for (int j = 0; j < n; ++j) {
-        float4 vv;
-        if (VQ) {
-            vv = vq_decode4(reinterpret_cast<const uint8_t *>(vb + j * kRowBytes), lane);
-        } else if (DT == SIKV_DTYPE_BF16) {
-            const uint2 w = *reinterpret_cast<const uint2 *>(vb + j * kRowBytes + 8 * lane);
-            vv = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-        } else {
-            vv = *reinterpret_cast<const float4 *>(vb + j * kRowBytes + 16 * lane);
-        }
-#pragma unroll
-        for (int g = 0; g < GM; ++g) {
-            const float w = __shfl_sync(0xffffffffu, pr[g], j0 + j);
-            s.o[g][0] = fmaf(w, vv.x, s.o[g][0]);
-            s.o[g][1] = fmaf(w, vv.y, s.o[g][1]);
-            s.o[g][2] = fmaf(w, vv.z, s.o[g][2]);
-            s.o[g][3] = fmaf(w, vv.w, s.o[g][3]);
-        }
-    }
-}
-
-// Winners among many candidates (more than the rank path takes): radix
-// select of the need-th key and of the lowest tied token indices, then one
-// marking pass.  Returns this thread's count of winners before the chunk.
-// Kept out of line: it only runs for heavily tied or flat score tables.
-__device__ __noinline__ uint32_t refine_by_radix(const uint2 *cand, int ncand, uint32_t need, int t0, int chunk,
-                                                 uint32_t *winbits, uint32_t *hist, uint32_t *wtot, uint32_t *sc) {
-    uint32_t ties_needed, left, before = 0;
-    const uint32_t T = cta_radix_select([&](int e) { return __ldcg(cand + e).x; }, [&](int) { return true; }, ncand,
-                                        need, hist, wtot, sc, &ties_needed);
-    // the ties_needed lowest token indices among keys equal to T
-    const uint32_t tie_idx = ~cta_radix_select([&](int e) { return ~__ldcg(cand + e).y; },
-                                               [&](int e) { return __ldcg(cand + e).x == T; }, ncand, ties_needed,
-                                               hist, wtot, sc, &left);
-    for (int e = threadIdx.x; e < ncand; e += kFT) {
-        const uint2 v = __ldcg(cand + e);
-        if (v.x > T || (v.x == T && v.y <= tie_idx)) {
-            const int rel = static_cast<int>(v.y) - t0;
-            if (rel >= 0 && rel < chunk) atomicOr(&winbits[rel >> 5], 1u << (rel & 31));
-            else if (rel < 0) ++before;
-        }
-    }
-    return before;
-}
 
 template <int DT, int GM, bool VQ>
 __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
@@ -846,8 +536,8 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                     }
                 }
             } else {
-                win_before += refine_by_radix(cand, ncand, need, t0, a.chunk, sh.u.sel.winbits, sh.hist, sh.wtot,
-                                              sh.sc);
+                win_before += refine_by_radix([&](int e) { return __ldcg(cand + e); }, ncand, need, t0, a.chunk,
+                                              sh.u.sel.winbits, sh.hist, sh.wtot, sh.sc);
             }
             __syncthreads();
             // each warp lists the winners of its share of the chunk's bitmap,
@@ -1136,15 +826,19 @@ sikv_status launch_fused_t(const FusedArgs &args, const FusedPlan &plan, cudaStr
 
 // Per device: the kernel's dynamic shared-memory limit is raised once, and
 // its occupancy (CTAs per SM) is computed once.  Values are idempotent, so
-// concurrent first calls only repeat the same work.
+// concurrent first calls only repeat the same work and store the same value
+// (relaxed atomics: no data race).
 constexpr int kMaxDevices = 64;
 
 template <int DT, int GM, bool VQ>
 int occupancy_of() {
-    static int cached[kMaxDevices];            // 0: unknown, else occupancy + 1
+    static std::atomic<int> cached[kMaxDevices];    // 0: unknown, else occupancy + 1
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev] - 1;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c - 1;
+    }
     // the occupancy calculator honours the kernel's dynamic shared-memory
     // limit, which must be raised above the 48 KB default first
     auto kern = decode_fused_kernel<DT, GM, VQ>;
@@ -1154,7 +848,7 @@ int occupancy_of() {
     int blocks = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kFT, sizeof(FusedSmem<GM>)) != cudaSuccess)
         return 0;
-    if (dev >= 0 && dev < kMaxDevices) cached[dev] = blocks + 1;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev].store(blocks + 1, std::memory_order_relaxed);
     return blocks;
 }
 

@@ -351,6 +351,89 @@ def check_needle_recall(o):
     assert set(hi.needle_pos.tolist()) <= set(idx.tolist())
 
 
+
+# --------------------------------------------------------------------------
+# one decode step: score, select, attend (§2.1 items 2-4), composed
+# --------------------------------------------------------------------------
+
+def check_decode_step_golden(o):
+    """The composed step on the hand-worked D = 4 case with one sink.
+
+    k = 2 selects {1, 2} and reproduces the worked attention output; k = 3
+    selects {1, 2, 4}; a softmax scale of 1 instead of 1/sqrt(D) doubles the
+    logits.  Closed forms, worked by hand from the fixture's keys (token t's
+    reconstructed key is 2 e_{t-1} for t = 1..4, the sink's key is 0):
+      scale 1/2, k = 3: head 0 logits (0, 1, 0, 0) over tokens (0, 1, 2, 4)
+        -> [2, e + 1, 2, 1] / (3 + e); head 1 logits (0, 0, 1, 1)
+        -> [1 + e, 1 + e, 2 e, e] / (2 + 2 e);
+      scale 1, k = 2: head 0 -> [1, e^2, 1, 0] / (2 + e^2),
+        head 1 -> [1, 1, e^2, 0] / (2 + e^2)."""
+    case = _load("codebook_d4.json")["cases"][0]
+    K = np.asarray(case["keys"], dtype=np.float64)
+    V = np.asarray(case["values"], dtype=np.float64)
+    q = np.asarray(case["queries"], dtype=np.float64)
+    s = case["num_sinks"]
+    mu, code, cent, _ = o.encode_keys(K, s)
+    out, idx, sc, _ = o.decode_step(q, K, V, mu, cent, code, 2, s)
+    assert list(idx) == case["topk"]["2"]
+    assert np.isneginf(sc[0]) and np.allclose(sc[1:], case["scores"][1:], rtol=0, atol=1e-15)
+    assert np.allclose(out, case["attention_k2"]["out"], rtol=0, atol=1e-15), out
+    e = math.e
+    out3, idx3, _, _ = o.decode_step(q, K, V, mu, cent, code, 3, s)
+    assert list(idx3) == case["topk"]["3"]
+    want3 = np.array([[2, e + 1, 2, 1], [1 + e, 1 + e, 2 * e, e]]) / np.array([[3 + e], [2 + 2 * e]])
+    assert np.allclose(out3, want3, rtol=0, atol=1e-15), out3
+    out_s1, _, _, _ = o.decode_step(q, K, V, mu, cent, code, 2, s, scale=1.0)
+    e2 = math.exp(2.0)
+    want_s1 = np.array([[1, e2, 1, 0], [1, 1, e2, 0]]) / (2 + e2)
+    assert np.allclose(out_s1, want_s1, rtol=0, atol=1e-15), out_s1
+
+
+def _embed_d4_case(o, d=128):
+    """The D = 4 fixture embedded in D = 128: the extra key channels are 0
+    (their codes are all 15 and their centroids 0, so scores and logits are
+    unchanged) and the value rows get an exactly representable 2-bit grid."""
+    case = _load("codebook_d4.json")["cases"][0]
+    K4 = np.asarray(case["keys"], dtype=np.float64)
+    n = K4.shape[0]
+    K = np.zeros((n, d))
+    K[:, :4] = K4
+    q = np.zeros((2, d))
+    q[:, :4] = np.asarray(case["queries"], dtype=np.float64)
+    rng = np.random.default_rng(44)
+    grid = rng.integers(0, 4, (n, d)).astype(np.float64)
+    grid[:, ::32] = 0.0
+    grid[:, 1::32] = 3.0
+    V = 0.5 + 0.25 * grid
+    return case, K, V, q
+
+
+def check_decode_step_qv(o):
+    """The 2-bit step: with values on the exact 2-bit grid it equals the
+    full-precision step (selection included) for any k, sink count and
+    scale; with off-grid values the selection is unchanged and the output
+    moves by at most the largest read-back error of a selected row."""
+    case, K, V, q = _embed_d4_case(o)
+    s = case["num_sinks"]
+    mu, code, cent, _ = o.encode_keys(K, s)
+    packed = o.quantize_values(V)
+    for k, scale in ((2, None), (3, None), (2, 1.0), (4, 0.25)):
+        a, ia, _, _ = o.decode_step(q, K, V, mu, cent, code, k, s, scale)
+        b, ib, _, _ = o.decode_step_qv(q, K, V, packed, mu, cent, code, k, s, scale)
+        assert list(ia) == list(ib) == sorted(case["topk"][str(k)])
+        assert np.allclose(a, b, rtol=0, atol=1e-15)
+    rng = np.random.default_rng(45)
+    Vr = rng.standard_normal(V.shape).astype(np.float32).astype(np.float64)
+    pr = o.quantize_values(Vr)
+    a, ia, _, _ = o.decode_step(q, K, Vr, mu, cent, code, 3, s, 1.0)
+    b, ib, _, _ = o.decode_step_qv(q, K, Vr, pr, mu, cent, code, 3, s, 1.0)
+    worst = np.abs(o.dequantize_values(pr) - Vr)[ia].max()
+    assert list(ia) == list(ib) and np.all(np.abs(a - b) <= worst + 1e-12)
+    assert not np.allclose(a, b, rtol=0, atol=1e-9)
+    # with nothing selected only the full-precision sink is attended
+    c, _, _, _ = o.decode_step_qv(q, K, Vr, pr, mu, cent, code, 0, s)
+    assert np.allclose(c, Vr[0][None, :].repeat(2, 0), rtol=0, atol=1e-15)
+
 # --------------------------------------------------------------------------
 # decode-time append (R19, R20: frozen prefill mean and codebook)
 # --------------------------------------------------------------------------
@@ -615,7 +698,7 @@ ALL_CHECKS = [
     check_codes_by_construction, check_codebook_golden, check_codebook_invariants,
     check_one_member_clusters_reconstruct, check_scores_golden, check_lut_identity,
     check_topk, check_attention_golden, check_attention_full_selection_is_dense,
-    check_attention_invariants, check_needle_recall, check_append_by_construction, check_append_golden,
+    check_attention_invariants, check_needle_recall, check_decode_step_golden, check_decode_step_qv, check_append_by_construction, check_append_golden,
     check_dense_scores_equal_lut_scores_when_exact, check_dense_attention,
     check_kmeans_golden, check_kmeans_update_exact, check_kmeans_matches_sklearn,
     check_kmeans_lloyd_invariants, check_values_golden, check_values_error_bound, check_values_attention,

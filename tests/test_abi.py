@@ -175,3 +175,27 @@ def test_value_quantization_entry_points_validate_without_launch():
     wa = L.sikv_sparse_attn_workspace_size(ctypes.byref(p))
     assert L.sikv_sparse_attn_qv(ctypes.byref(p), fake, fake, fake, None, *args[:7], fake, wa, None) == 1
     assert L.sikv_sparse_attn_qv(ctypes.byref(p), fake, fake, fake, odd, *args[:7], fake, wa, None) == 2
+
+
+def test_static_attention_entry_validates_without_launch():
+    """sikv_sparse_attn_static refuses null or misaligned pointers, invalid
+    parameters and sizes beyond its fixed scratch array on the host, before
+    it looks up the array or launches anything."""
+    fn = sk.lib().sikv_sparse_attn_static
+    fn.argtypes = [ctypes.POINTER(sk.Params)] + [ctypes.c_void_p] * 12
+    fn.restype = ctypes.c_int
+    p = _p()
+    fake = ctypes.c_void_p(1 << 20)
+    null = ctypes.c_void_p(0)
+    args = [fake] * 10                       # q, K, V, codes, codebook, mu, idx, k_per_seq, seq_lens, out
+    assert fn(ctypes.byref(p), null, *args[1:], null, null) == 1          # null q
+    assert fn(ctypes.byref(p), *args[:9], null, null, null) == 1          # null out
+    assert fn(ctypes.byref(p), *args[:6], null, *args[7:], null, null) == 1   # null idx with kmax > 0
+    bad = _p(num_q_heads=7)
+    assert fn(ctypes.byref(bad), *args, null, null) == 1                  # invalid parameters
+    odd16 = ctypes.c_void_p((1 << 20) + 8)
+    assert fn(ctypes.byref(p), odd16, *args[1:], null, null) == 2          # q not 16-byte aligned
+    odd4 = ctypes.c_void_p((1 << 20) + 2)
+    assert fn(ctypes.byref(p), *args, odd4, null) == 2                    # device_flags not 4-byte aligned
+    big = sk.make_params("bf16", 256, 32, 8, 131072, 64, 2048)
+    assert fn(ctypes.byref(big), *args, null, null) == 3                  # partials beyond the 8 MiB array

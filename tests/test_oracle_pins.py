@@ -162,6 +162,27 @@ def _mut_values_sinks_quantized(q_group, K, V, packed, mu, centroids, code, idx,
     return oracle.sparse_attention(q_group, K, Vq, mu, centroids, code, idx, num_sinks, scale)
 
 
+
+def _mut_decode_drops_sinks(q_group, K, V, mu, centroids, code, k, num_sinks=64, scale=None):
+    sc, cond = oracle.scores(q_group, mu, centroids, code, num_sinks)
+    idx = oracle.topk(sc, k, num_sinks)
+    return oracle.sparse_attention(q_group, K, V, mu, centroids, code, idx, scale=scale), idx, sc, cond
+
+
+def _mut_decode_drops_scale(q_group, K, V, mu, centroids, code, k, num_sinks=64, scale=None):
+    return oracle.decode_step(q_group, K, V, mu, centroids, code, k, num_sinks)
+
+
+def _mut_decode_qv_drops_sinks(q_group, K, V, packed, mu, centroids, code, k, num_sinks=64, scale=None):
+    sc, cond = oracle.scores(q_group, mu, centroids, code, num_sinks)
+    idx = oracle.topk(sc, k, num_sinks)
+    out = oracle.sparse_attention_qv(q_group, K, V, packed, mu, centroids, code, idx, scale=scale)
+    return out, idx, sc, cond
+
+
+def _mut_decode_qv_drops_scale(q_group, K, V, packed, mu, centroids, code, k, num_sinks=64, scale=None):
+    return oracle.decode_step_qv(q_group, K, V, packed, mu, centroids, code, k, num_sinks)
+
 MUTATIONS = {
     "strict-greater": dict(sign_codes=_mut_codes_strict),
     "msb-first-bits": dict(sign_codes=_mut_codes_msb_first),
@@ -186,6 +207,10 @@ MUTATIONS = {
     "values-levels-msb-first": dict(quantize_values=_mut_values(msb_first=True)),
     "values-groups-of-16": dict(quantize_values=_mut_values(group=16)),
     "values-sinks-quantized": dict(sparse_attention_qv=_mut_values_sinks_quantized),
+    "decode-drops-num-sinks": dict(decode_step=_mut_decode_drops_sinks),
+    "decode-drops-scale": dict(decode_step=_mut_decode_drops_scale),
+    "decode-qv-drops-num-sinks": dict(decode_step_qv=_mut_decode_qv_drops_sinks),
+    "decode-qv-drops-scale": dict(decode_step_qv=_mut_decode_qv_drops_scale),
 }
 
 

@@ -7,7 +7,8 @@ They cannot pass the workspace that sikv_sparse_attn needs, so the library
 offers a variant whose scratch lives in a fixed 8 MiB array compiled into the
 library.  These tests call that variant through the C ABI and check that it
 returns what sikv_sparse_attn returns, on two calls in a row (the array keeps
-the previous call's contents), that it reports device-side errors, and that
+the previous call's contents) and what the oracle's attention gives over the
+same selection, that it reports device-side errors, and that
 sizes beyond its limit are refused before anything is launched.
 
 This file sorts last so that a run stopping at the first failure has already
@@ -21,6 +22,7 @@ import pytest
 import torch
 
 import long_context_decode_sikv_b200 as sk
+import oracle
 import sikv_inputs as gen
 from tests import gpu_util as gu
 
@@ -58,6 +60,7 @@ def test_static_scratch_matches_workspace_variant_twice():
     flags = torch.full((1,), -1, dtype=torch.int32, device=dev)
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     atol, rtol = gu.attn_tol(w.dtype)
+    heads = {(b, h): gu.oracle_head(w, dw.bt, b, h) for b in range(w.batch) for h in range(w.num_kv_heads)}
     for step in (0, 1):
         ref = torch.empty((w.batch, w.num_q_heads, 128), dtype=dw.p.torch_dtype, device=dev)
         sk.sikv_sparse_attn(dw.p, dw.q[step], dw.K, dw.V, c.codes, c.codebook, c.mu, idx, dw.k, dw.seq_lens,
@@ -70,6 +73,17 @@ def test_static_scratch_matches_workspace_variant_twice():
         assert flags.item() == 0
         assert torch.isfinite(out.float()).all()
         assert np.allclose(gu.to_f64(out), gu.to_f64(ref), atol=atol, rtol=rtol), step
+        # and directly against the oracle's attention over the same selection
+        got = gu.to_f64(out)
+        idx_h = idx.cpu().numpy()
+        for b in range(w.batch):
+            k = w.topk[b]
+            for h in range(w.num_kv_heads):
+                o = heads[(b, h)]
+                q = gu.oracle_queries(w, dw.bt, step, b, h)
+                want = oracle.sparse_attention(q, o.K, o.V, o.mu, o.cent, o.code, idx_h[b, h, :k], w.num_sinks)
+                g = got[b, h * w.group:(h + 1) * w.group]
+                assert np.allclose(g, want, atol=atol, rtol=rtol), (step, b, h, float(np.abs(g - want).max()))
 
 
 def test_static_scratch_reports_device_errors():
