@@ -43,8 +43,13 @@ UNIT = "decode steps/s"
 PROFILED = {
     "score": ("score_kernel_long_context_b4_n131072.md", ("score_device.cuh", "score.cu", "sikv_common.cuh")),
     "decode_fused": ("decode_fused_kernel_long_context_b4_n131072.md",
-                     ("score_device.cuh", "decode_fused.cu", "sikv_common.cuh")),
+                     ("score_device.cuh", "decode_common.cuh", "decode_fused.cu", "sikv_common.cuh")),
+    "decode_cluster": ("decode_cluster_kernel_long_context_b4_n131072.md",
+                       ("score_device.cuh", "decode_common.cuh", "decode_cluster.cu", "sikv_common.cuh")),
 }
+KERNEL_OF_PATH = {1: ("decode_cluster", "decode_cluster_kernel (score + top-k + sparse attention, one cluster "
+                                        "per segment)"),
+                  2: ("decode_fused", "decode_fused_kernel (score + top-k + sparse attention, cooperative)")}
 
 
 def parse_args(argv=None):
@@ -58,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extreme-encode", action="store_true", help="skip the 512K-key encoder leg")
+    ap.add_argument("--no-all-core-oracle", action="store_true", help="skip the all-core oracle figure")
     return ap.parse_args(argv)
 
 
@@ -279,23 +286,83 @@ def oracle_decode_seconds(w: gen.Workload, budget_s: float, max_iters: int, toke
     return per_seg * w.segments, desc, 1, times
 
 
+def _oracle_steps_worker(cfg, segs, warmup, steps, start, results):
+    """One worker process of the whole-step oracle run: regenerates and
+    encodes its segments (not timed), then decodes them for every step with
+    that step's query, single-threaded, timing the ``steps`` steps after the
+    common start barrier."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+
+    w = gen.config(cfg)
+    data = []
+    for (b, h) in segs:
+        hi = gen.head_inputs(w, b, h, steps=tuple(range(warmup + steps)))
+        K = gen.storage_to_f64(hi.keys, w.dtype)
+        V = gen.storage_to_f64(hi.values, w.dtype)
+        mu, code, cent, _ = oracle.encode_keys(K, w.num_sinks)
+        qs = [gen.storage_to_f64(hi.queries[i], w.dtype) for i in range(warmup + steps)]
+        data.append((K, V, mu, code, cent, qs, w.topk[b]))
+    with threadpool_limits(limits=1):
+        for i in range(warmup):
+            for (K, V, mu, code, cent, qs, k) in data:
+                oracle.decode_step(qs[i], K, V, mu, cent, code, k, w.num_sinks)
+        start.wait()
+        t0 = time.perf_counter()
+        for i in range(warmup, warmup + steps):
+            for (K, V, mu, code, cent, qs, k) in data:
+                oracle.decode_step(qs[i], K, V, mu, cent, code, k, w.num_sinks)
+        results.put(time.perf_counter() - t0)
+
+
+def oracle_whole_steps(cfg: int, steps: int, warmup: int, max_workers: int | None = None):
+    """The oracle on whole decode steps (every segment of the batch, the query
+    redrawn every step), its segments spread over spawned worker processes,
+    one single-threaded worker per available core (at most one per segment).
+
+    Returns (seconds per step, workers, description).  The step time is the
+    slowest worker's time over the timed steps divided by their number: a
+    step is done when its last segment is."""
+    import multiprocessing as mp
+
+    w = gen.config(cfg)
+    cores = len(os.sched_getaffinity(0))
+    segs = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+    workers = max(1, min(cores, len(segs), max_workers or len(segs)))
+    parts = [segs[i::workers] for i in range(workers)]
+    ctx = mp.get_context("spawn")
+    start = ctx.Barrier(workers)
+    results = ctx.Queue()
+    procs = [ctx.Process(target=_oracle_steps_worker, args=(cfg, part, warmup, steps, start, results))
+             for part in parts]
+    for pr in procs:
+        pr.start()
+    elapsed = [results.get() for _ in procs]
+    for pr in procs:
+        pr.join()
+    per_step = max(elapsed) / steps
+    desc = (f"oracle decode_step (fp64 numpy, single-threaded per process) on whole steps: all "
+            f"{len(segs)} (sequence, KV head) segments of the workload, {steps} timed steps after {warmup} "
+            f"warm-up, queries redrawn every step; segments spread over {workers} worker processes "
+            f"({cores} cores available)")
+    return per_step, workers, desc
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     w = gen.config(args.config)
-    total = args.steps + args.warmup
-    budget = 150.0
-    # one full segment takes ~0.1 s on one core: shrink the token sample for long runs
-    frac = min(1.0, (budget / max(total, 1)) / 0.12)
-    per_step, desc, cores, times = oracle_decode_seconds(w, budget_s=budget, max_iters=total, token_frac=frac)
+    steps, warmup = max(1, args.steps), max(0, min(args.warmup, 2))
+    per_step, workers, desc = oracle_whole_steps(args.config, steps, warmup)
     value = 1.0 / per_step
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": len(times),
-        "warmup": 0, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": steps,
+        "warmup": warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, replicas=0),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": desc,
+                         "cores_available": len(os.sched_getaffinity(0))},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -351,6 +418,7 @@ def run_sikv(args):
     torch.cuda.synchronize()
     enc_ms = e0.elapsed_time(e1) / 3
     base.check()
+    k_bytes = K.numel() * K.element_size()
 
     # replicas of the encoded cache so that no step's inputs sit in L2
     sb = step_bytes(w)
@@ -419,10 +487,38 @@ def run_sikv(args):
     g_dec = graph_of(decode_step, args.warmup, total)
     sampler = ClockSampler(dev)
     with sampler:
-        ms = timed(g_dec)
+        reps_ms = [max_over_ranks(timed(g_dec), world) for _ in range(5)]
     ws.check()
-    ms = max_over_ranks(ms, world)
+    ms = statistics.median(reps_ms)
     del g_dec
+    # the graph's last step left its output in `out`: an eager call on the
+    # same query and replica must give the same bytes
+    graph_out = out.clone()
+    with torch.cuda.stream(stream):
+        decode_step(total - 1)
+    torch.cuda.synchronize()
+    last_step_identical = bool(torch.equal(graph_out, out))
+
+    # the other single-launch kernel on the same steps, for comparison
+    resolved = int(sk.lib().sikv_decode_resolved_path(ctypes.byref(p)))
+    alt_ms, alt_name = None, None
+    alt_path = 2 if resolved == 1 else (1 if resolved == 2 else 0)
+    if alt_path:
+        p_alt = sk.make_params(w.dtype, w.batch, w.num_q_heads, w.num_kv_heads, w.max_seq_len, w.num_sinks,
+                               w.max_topk, decode_path=alt_path)
+        if int(sk.lib().sikv_decode_resolved_path(ctypes.byref(p_alt))) == alt_path:
+            def alt_step(i):
+                c = reps[i % R]
+                sk.sikv_decode(p_alt, qs[i], c.K, c.V, c.codes, c.codebook, c.mu, seq, kk, out, workspace=ws)
+
+            with torch.cuda.stream(stream):
+                for i in range(args.warmup):
+                    alt_step(i)
+            g = graph_of(alt_step, args.warmup, total)
+            alt_ms = max_over_ranks(timed(g), world)
+            alt_name = KERNEL_OF_PATH[alt_path][0]
+            del g
+            ws.check()
 
     # per-kernel breakdown over the same steps (dominant kernel timed live)
     torch.cuda.synchronize()
@@ -540,7 +636,16 @@ def run_sikv(args):
     barrier(world)
     km_ms = max_over_ranks(a.elapsed_time(b), world) / 2
     ws_km.check()
+    # bound-based: per k-means iteration the assignment reads K and writes the
+    # codes, the accumulation reads K and the codes; the one-pass encoder
+    # reads K twice (mean, then codes and cluster sums) and writes the codes
+    kb, cb_ = K.numel() * K.element_size(), base.codes.numel()
+    hbm = float(measured_peaks()[0]["hbm_gbs"]) * 1e9
+    km_bound_ms = 20 * (2 * kb + 2 * cb_) / hbm * 1e3
+    enc_bound_ms = (2 * kb + cb_) / hbm * 1e3
     comparison.update({
+        "kmeans20_roofline_ms": km_bound_ms, "one_pass_encode_roofline_ms": enc_bound_ms,
+        "clustering_speedup_roofline": km_bound_ms / enc_bound_ms,
         "one_pass_encode_ms": enc_ms, "kmeans20_ms": km_ms,
         "clustering_speedup_one_pass_vs_kmeans20": km_ms / enc_ms,
         "kmeans_iteration_us": 1e3 * km_ms / 20,
@@ -581,6 +686,44 @@ def run_sikv(args):
                "api": "sikv_decode_host (C ABI) on page-locked host buffers, one call per step; the "
                       "kernels read the query and write the output over the host link"}
 
+    # prefill encoder at the extreme-context shape (B=1, 32/8 heads, 512K keys
+    # per head, the same generator with drift): keys encoded per second over
+    # all 512K x 8 keys, and GB/s over its algorithmic bytes (two reads of K
+    # plus the code rows written)
+    encode_extreme = None
+    if args.config == 2 and world == 1 and not args.no_extreme_encode:
+        from concurrent.futures import ThreadPoolExecutor
+
+        del reps, base, K, V
+        torch.cuda.empty_cache()
+        w4 = gen.config(4)
+        n4 = w4.max_seq_len
+        with ThreadPoolExecutor(min(8, os.cpu_count() or 1)) as ex:
+            keys = list(ex.map(lambda h: gen.head_inputs(w4, 0, h).keys, range(w4.num_kv_heads)))
+        K4 = sk.to_device(np.stack(keys)[None], w4.dtype, dev)
+        del keys
+        p4 = sk.make_params(w4.dtype, 1, w4.num_q_heads, w4.num_kv_heads, n4, w4.num_sinks, w4.max_topk)
+        c4 = sk.SikvCache(p4, K4, K4, torch.full((1,), n4, dtype=torch.int32, device=dev))
+        c4.encode()
+        torch.cuda.synchronize()
+        a4, b4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a4.record()
+        for _ in range(3):
+            c4.encode()
+        b4.record()
+        torch.cuda.synchronize()
+        c4.check()
+        ms4 = a4.elapsed_time(b4) / 3
+        keys4 = w4.num_kv_heads * n4
+        bytes4 = 2 * K4.numel() * K4.element_size() + c4.codes.numel()
+        encode_extreme = {"workload": w4.name, "keys": keys4, "ms": ms4, "keys_per_s": keys4 / (ms4 / 1e3),
+                          "GB_per_s": bytes4 / (ms4 / 1e3) / 1e9,
+                          "frac_of_hbm": bytes4 / (ms4 / 1e3) / 1e9 / float(measured_peaks()[0]["hbm_gbs"]),
+                          "algorithmic_bytes": bytes4,
+                          "note": "mean, sign codes and one-pass codebook of every key (sikv_encode_keys)"}
+        del c4, K4
+        torch.cuda.empty_cache()
+
     peaks, peak_src = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     score_launch_s = ms_score / 1e3 / args.steps
@@ -588,12 +731,13 @@ def run_sikv(args):
     step_s = ms / 1e3 / args.steps
     step_gbs = sb / step_s / 1e9
     launches = int(sk.lib().sikv_decode_launches(ctypes.byref(p)))
-    if launches == 1:
-        # one cooperative kernel per step: the timed graph holds exactly one
+    if launches == 1 and resolved in KERNEL_OF_PATH:
+        # one single-launch kernel per step: the timed graph holds exactly one
         # launch per step, so its average duration is the step time
-        roofline = {"bound": "hbm", "kernel": "decode_fused_kernel (score + top-k + sparse attention)",
+        kname, kdesc = KERNEL_OF_PATH[resolved]
+        roofline = {"bound": "hbm", "kernel": kdesc,
                     "achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
-                    "traffic": profiled_traffic("decode_fused"), "algorithmic_bytes_per_launch": sb,
+                    "traffic": profiled_traffic(kname), "algorithmic_bytes_per_launch": sb,
                     "peak_source": f"{peak_src} hbm_gbs (copy, of measured)"}
     else:
         roofline = {"bound": "hbm", "kernel": "score_kernel (LUT-GEMV scoring)", "achieved": score_gbs,
@@ -614,20 +758,29 @@ def run_sikv(args):
                           "algorithmic_bytes_per_step": sb,
                           "formula": "per (seq, kv head): 16*(N-S) code bytes + k*D*2 V bytes + S*2*D*2 sink "
                                      "K/V bytes + 8 KB codebook"},
+        "timed_replays": {"runs": len(reps_ms), "ms_per_step_median": ms / args.steps,
+                          "ms_per_step_min": min(reps_ms) / args.steps, "ms_per_step_max": max(reps_ms) / args.steps,
+                          "last_step_output_identical_to_eager_call": last_step_identical},
         "breakdown_us_per_step": {"decode": 1e3 * ms / args.steps, "score": 1e3 * ms_score / args.steps,
-                                  "topk": 1e3 * ms_topk / args.steps, "sparse_attn": 1e3 * ms_attn / args.steps},
+                                  "topk": 1e3 * ms_topk / args.steps, "sparse_attn": 1e3 * ms_attn / args.steps,
+                                  **({f"decode_{alt_name}": 1e3 * alt_ms / args.steps} if alt_ms else {})},
         "encode": {"ms": enc_ms, "keys_per_s": w.batch * w.num_kv_heads * w.max_seq_len / (enc_ms / 1e3),
-                   "GB_per_s_2reads": 2 * K.numel() * K.element_size() / (enc_ms / 1e3) / 1e9},
+                   "GB_per_s_2reads": 2 * k_bytes / (enc_ms / 1e3) / 1e9},
         "comparison": comparison,
         "values_2bit": values_2bit,
         "clocks": sampler.summary(),
         "gpu_launches": launches * args.steps,
         "e2e": e2e,
+        "encode_extreme_context": encode_extreme,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per_step, desc, cores, times = oracle_decode_seconds(w, args.cpu_seconds, 10_000)
         line["cpu_baseline"] = {"value": 1.0 / per_step, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "cores_available": len(os.sched_getaffinity(0))}
+        if not args.no_all_core_oracle:
+            per_all, workers, desc_all = oracle_whole_steps(args.config, steps=2, warmup=1)
+            line["cpu_baseline"]["all_cores"] = {"value": 1.0 / per_all, "unit": UNIT, "cores": workers,
+                                                 "sample": desc_all}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

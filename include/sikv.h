@@ -106,8 +106,31 @@ typedef struct sikv_params {
     int32_t num_sinks;      /* S >= 0 (the pages keep 64) */
     int32_t max_topk;       /* kmax >= 0: row capacity of idx */
     float softmax_scale;    /* <= 0 selects 1/sqrt(D) */
-    int32_t reserved[3];    /* must be 0 */
+    int32_t decode_path;    /* sikv_decode_path: which kernels sikv_decode runs (0: automatic) */
+    int32_t reserved[2];    /* must be 0 */
 } sikv_params;
+
+/*
+ * Kernels of one sikv_decode / sikv_decode_qv / sikv_decode_host step.  Every
+ * path computes the same result (identical scores, identical selection; the
+ * attention differs only by fp32 summation order).  AUTO picks the first that
+ * applies to the shape, in this order; a forced path that does not apply
+ * returns SIKV_ERR_UNSUPPORTED.
+ *  - CLUSTER: one launch; the CTAs of each (sequence, KV head) segment form a
+ *    thread-block cluster (at most 16 CTAs of 16384 tokens: Nmax <= 262144)
+ *    and agree through distributed shared memory.  Any batch size: clusters
+ *    that do not fit at once run in later waves.
+ *  - COOPERATIVE: one cooperative launch per group of sequences whose CTAs all
+ *    fit on the device at once; the CTAs of a segment agree through counters
+ *    in the workspace.  Any Nmax.
+ *  - COMPOSED: sikv_score, sikv_topk and sikv_sparse_attn's kernels.
+ */
+typedef enum sikv_decode_path {
+    SIKV_DECODE_AUTO = 0,
+    SIKV_DECODE_CLUSTER = 1,
+    SIKV_DECODE_COOPERATIVE = 2,
+    SIKV_DECODE_COMPOSED = 3
+} sikv_decode_path;
 
 /* Library version as 10000*major + 100*minor + patch. */
 SIKV_API int32_t sikv_version(void);
@@ -136,8 +159,14 @@ SIKV_API size_t sikv_kmeans_workspace_size(const sikv_params *p);
 SIKV_API size_t sikv_quantize_values_workspace_size(const sikv_params *p);
 
 /* Number of kernels one sikv_decode call enqueues for these parameters
- * (0 on bad params). */
+ * (0 on bad params, or when the forced decode_path does not apply). */
 SIKV_API int32_t sikv_decode_launches(const sikv_params *p);
+
+/* The sikv_decode_path (CLUSTER, COOPERATIVE or COMPOSED) that one
+ * sikv_decode call with these parameters runs on the current device: the
+ * automatic choice resolved, or the forced path; 0 on bad params or when a
+ * forced path does not apply.  Queries occupancy once per device. */
+SIKV_API int32_t sikv_decode_resolved_path(const sikv_params *p);
 
 /*
  * sikv_encode_keys -- prefill encoder [SIKV 2.1.1, 2.1.3].

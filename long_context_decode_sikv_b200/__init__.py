@@ -15,7 +15,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from ._binding import (EXPORTED, SIKV_DEVERR_APPEND, SIKV_DEVERR_INDEX, SIKV_DEVERR_SEQ_LEN,  # noqa: F401
+from ._binding import (EXPORTED, SIKV_DECODE_AUTO, SIKV_DECODE_CLUSTER, SIKV_DECODE_COMPOSED,  # noqa: F401
+                       SIKV_DECODE_COOPERATIVE, SIKV_DEVERR_APPEND, SIKV_DEVERR_INDEX, SIKV_DEVERR_SEQ_LEN,  # noqa: F401
                        SIKV_DEVERR_TOPK, SIKV_DTYPE_BF16, SIKV_DTYPE_F32, DecodeHostPlan, Params, SikvError,
                        Workspace, default_scale, lib, library_path, make_params, sikv_append_codes, sikv_decode,
                        sikv_decode_host, sikv_dense_attn, sikv_dense_score, sikv_encode_keys, sikv_kmeans_codebook,

@@ -27,6 +27,12 @@ SIKV_DEVERR_INDEX = 0x4
 SIKV_DEVERR_TIMEOUT = 0x8
 SIKV_DEVERR_APPEND = 0x10
 
+# sikv_params.decode_path: which kernels a decode step runs
+SIKV_DECODE_AUTO = 0
+SIKV_DECODE_CLUSTER = 1
+SIKV_DECODE_COOPERATIVE = 2
+SIKV_DECODE_COMPOSED = 3
+
 _STATUS = {0: "SIKV_OK", 1: "SIKV_ERR_INVALID_ARG", 2: "SIKV_ERR_UNSUPPORTED", 3: "SIKV_ERR_WORKSPACE",
            4: "SIKV_ERR_CUDA", 5: "SIKV_ERR_DEVICE"}
 
@@ -34,6 +40,7 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_encode_workspace_size", "sikv_score_workspace_size", "sikv_topk_workspace_size",
             "sikv_sparse_attn_workspace_size", "sikv_decode_workspace_size", "sikv_encode_keys",
             "sikv_score", "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_launches",
+            "sikv_decode_resolved_path",
             "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
             "sikv_append_workspace_size", "sikv_append_codes", "sikv_dense_attn_workspace_size",
             "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_workspace_size", "sikv_kmeans_codebook",
@@ -58,7 +65,7 @@ class Params(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int32), ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
                 ("num_sinks", ctypes.c_int32), ("max_topk", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
-                ("reserved", ctypes.c_int32 * 3)]
+                ("decode_path", ctypes.c_int32), ("reserved", ctypes.c_int32 * 2)]
 
     @property
     def group(self) -> int:
@@ -74,13 +81,14 @@ class Params(ctypes.Structure):
 
 
 def make_params(dtype, batch, num_q_heads, num_kv_heads, max_seq_len, num_sinks=64, max_topk=0,
-                head_dim=128, softmax_scale=0.0) -> Params:
+                head_dim=128, softmax_scale=0.0, decode_path=0) -> Params:
     if isinstance(dtype, str):
         dtype = {"f32": SIKV_DTYPE_F32, "bf16": SIKV_DTYPE_BF16}[dtype]
     elif isinstance(dtype, torch.dtype):
         dtype = {torch.float32: SIKV_DTYPE_F32, torch.bfloat16: SIKV_DTYPE_BF16}[dtype]
     return Params(int(dtype), int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), int(max_seq_len),
-                  int(num_sinks), int(max_topk), float(softmax_scale), (ctypes.c_int32 * 3)(0, 0, 0))
+                  int(num_sinks), int(max_topk), float(softmax_scale), int(decode_path),
+                  (ctypes.c_int32 * 2)(0, 0))
 
 
 _LIB = None
@@ -109,6 +117,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, n).argtypes = [pp]
         L.sikv_decode_launches.restype = i32
         L.sikv_decode_launches.argtypes = [pp]
+        L.sikv_decode_resolved_path.restype = i32
+        L.sikv_decode_resolved_path.argtypes = [pp]
         L.sikv_encode_keys.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_score.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_topk.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]

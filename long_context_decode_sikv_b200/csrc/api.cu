@@ -23,13 +23,34 @@ sikv_status check_params(const sikv_params *p) {
     if (p->num_q_heads % p->num_kv_heads != 0) return SIKV_ERR_INVALID_ARG;
     if (p->num_q_heads / p->num_kv_heads > kMaxGroup) return SIKV_ERR_UNSUPPORTED;
     if (p->max_seq_len < 1 || p->num_sinks < 0 || p->max_topk < 0) return SIKV_ERR_INVALID_ARG;
-    if (p->reserved[0] || p->reserved[1] || p->reserved[2]) return SIKV_ERR_INVALID_ARG;
+    if (p->decode_path < SIKV_DECODE_AUTO || p->decode_path > SIKV_DECODE_COMPOSED) return SIKV_ERR_INVALID_ARG;
+    if (p->reserved[0] || p->reserved[1]) return SIKV_ERR_INVALID_ARG;
     if (!(p->softmax_scale <= 0.f || isfinite(p->softmax_scale))) return SIKV_ERR_INVALID_ARG;
     const long long segs = static_cast<long long>(p->batch) * p->num_kv_heads;
     if (segs > 65535) return SIKV_ERR_UNSUPPORTED;                      // grid.y limit
     if (static_cast<long long>(p->max_seq_len) > (1ll << 30)) return SIKV_ERR_UNSUPPORTED;
     if (static_cast<long long>(p->num_sinks) + p->max_topk > (1ll << 30)) return SIKV_ERR_UNSUPPORTED;
     return SIKV_OK;
+}
+
+// The kernels a decode step runs (sikv_decode_path; 0 when a forced path
+// does not apply).  The automatic choice follows measurements on B200: the
+// cooperative kernel when one launch covers the batch, except for segments
+// that a cluster of at most two CTAs covers (short contexts); the cluster
+// kernel when the cooperative one would need several launches (large ragged
+// batches); the three composed kernels otherwise.
+int resolve_decode_path(const sikv_params &p, bool vq) {
+    const int path = p.decode_path;
+    if (path == SIKV_DECODE_CLUSTER) return cluster_plan(p, vq).ok ? SIKV_DECODE_CLUSTER : 0;
+    if (path == SIKV_DECODE_COOPERATIVE)
+        return (fused_plan(p, vq).ok || fused_sub_batch(p, vq) > 0) ? SIKV_DECODE_COOPERATIVE : 0;
+    if (path == SIKV_DECODE_COMPOSED) return SIKV_DECODE_COMPOSED;
+    const ClusterPlan cp = cluster_plan(p, vq);
+    const bool single = fused_plan(p, vq).ok;
+    if (single && !(cp.ok && cp.csize <= 2)) return SIKV_DECODE_COOPERATIVE;
+    if (cp.ok) return SIKV_DECODE_CLUSTER;
+    if (fused_sub_batch(p, vq) > 0) return SIKV_DECODE_COOPERATIVE;
+    return SIKV_DECODE_COMPOSED;
 }
 
 sikv_status check_ws(void *ws, size_t bytes, size_t need) {
@@ -138,14 +159,27 @@ sikv_status decode_step(const sikv_params &pp, const void *q, const void *K, con
     char *ws = static_cast<char *>(workspace);
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     const bool qv = vq != nullptr;
-    const FusedPlan plan = fused_plan(*p, qv);
+    const int path = resolve_decode_path(*p, qv);
+    if (path == 0) return SIKV_ERR_UNSUPPORTED;
+    if (path == SIKV_DECODE_CLUSTER) {
+        const ClusterPlan cp = cluster_plan(*p, qv);
+        if (cp.ok) {
+            const FusedLayout FL = fused_layout(*p, L.fused);
+            return launch_decode_cluster(*p, cp, q, K, V, vq, codes, codebook, mu, seq_lens, k_per_seq, out, idx_out,
+                                         scores_out, reinterpret_cast<uint2 *>(ws + FL.cand), fused_cand_cap(*p),
+                                         status, s);
+        }
+        return SIKV_ERR_UNSUPPORTED;
+    }
+    const FusedPlan plan = path == SIKV_DECODE_COMPOSED ? FusedPlan() : fused_plan(*p, qv);
     if (plan.ok)
         return launch_decode_fused(*p, plan, fused_layout(*p, L.fused), q, K, V, vq, codes, codebook, mu, seq_lens,
                                    k_per_seq, out, idx_out, scores_out, ws, status, s);
     // Too many segments for one co-resident launch: run the single-launch
     // kernel on sub-batches of sequences that fit, one after the other on the
     // stream (each launch leaves the coordination state zeroed for the next).
-    const int bsub = fused_sub_batch(*p, qv);
+    const int bsub = path == SIKV_DECODE_COMPOSED ? 0 : fused_sub_batch(*p, qv);
+    if (path == SIKV_DECODE_COOPERATIVE && bsub == 0) return SIKV_ERR_UNSUPPORTED;
     if (bsub > 0) {
         // one coordination layout, the largest sub-batch's, for every
         // sub-launch: a layout sized by each launch's own batch would place
@@ -324,12 +358,23 @@ size_t sikv_decode_host_workspace_size(const sikv_params *p) {
     return sikv::host_layout(*p, decode_layout(*p).total).total;
 }
 
+int32_t sikv_decode_resolved_path(const sikv_params *p) {
+    if (check_params(p) != SIKV_OK) return 0;
+    return resolve_decode_path(*p, false);
+}
+
 int32_t sikv_decode_launches(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
-    if (fused_plan(*p).ok) return 1;               // one cooperative kernel
-    const int bsub = fused_sub_batch(*p);
-    if (bsub > 0) return (p->batch + bsub - 1) / bsub;   // one per sub-batch
-    return 1 + (p->max_topk > 0 ? 1 : 0) + 2;     // score, top-k, attention partials + combine
+    switch (resolve_decode_path(*p, false)) {
+        case SIKV_DECODE_CLUSTER: return 1;                      // one cluster launch
+        case SIKV_DECODE_COOPERATIVE: {
+            if (fused_plan(*p).ok) return 1;                     // one cooperative kernel
+            const int bsub = fused_sub_batch(*p);
+            return (p->batch + bsub - 1) / bsub;                 // one per sub-batch
+        }
+        case SIKV_DECODE_COMPOSED: return 1 + (p->max_topk > 0 ? 1 : 0) + 2;   // score, top-k, attention + combine
+        default: return 0;
+    }
 }
 
 sikv_status sikv_encode_keys(const sikv_params *p, const void *K, const int32_t *seq_lens, float *mu,

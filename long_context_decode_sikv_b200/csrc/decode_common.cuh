@@ -33,8 +33,11 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// Exclusive scan over the CTA (256 threads) of one value per thread.
+// Exclusive scan over the CTA (NT threads) of one value per thread; wtot
+// holds NT / 32 + 1 words.
+template <int NT = kFT>
 __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t *wtot, uint32_t *total) {
+    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t incl = v;
 #pragma unroll
@@ -46,28 +49,28 @@ __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t *wtot, ui
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t run = 0;
-        for (int w = 0; w < kFW; ++w) {
+        for (int w = 0; w < NW; ++w) {
             const uint32_t t = wtot[w];
             wtot[w] = run;
             run += t;
         }
-        wtot[kFW] = run;
+        wtot[NW] = run;
     }
     __syncthreads();
     const uint32_t r = wtot[warp] + incl - v;
-    *total = wtot[kFW];
+    *total = wtot[NW];
     __syncthreads();
     return r;
 }
 
-// In a histogram of PER * 256 bins scanned from the top bin down, finds the
+// In a histogram of PER * NT bins scanned from the top bin down, finds the
 // bin where the running count first reaches `need` (1 <= need <= total).
 // Each thread loads its PER consecutive bins once.  Writes (bin, count above)
 // to out[0..1]; out is left untouched when the total is below need.  Ends
 // synchronized.
-template <int PER, typename Load>
+template <int PER, int NT = kFT, typename Load>
 __device__ __forceinline__ void cta_find_bin(Load load, uint32_t need, uint32_t *wtot, uint32_t *out) {
-    const int top = PER * kFT - 1 - static_cast<int>(threadIdx.x) * PER;
+    const int top = PER * NT - 1 - static_cast<int>(threadIdx.x) * PER;
     uint32_t h[PER];
     uint32_t loc = 0;
 #pragma unroll
@@ -76,7 +79,7 @@ __device__ __forceinline__ void cta_find_bin(Load load, uint32_t need, uint32_t 
         loc += h[i];
     }
     uint32_t total;
-    uint32_t above = cta_excl_scan(loc, wtot, &total);
+    uint32_t above = cta_excl_scan<NT>(loc, wtot, &total);
     if (above < need && need <= above + loc) {
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
@@ -93,21 +96,26 @@ __device__ __forceinline__ void cta_find_bin(Load load, uint32_t need, uint32_t 
 // Radix select over `n` elements (element e has key key(e) and passes
 // keep(e)): returns the key of rank `need` counted from the largest and, in
 // *need_left, how many elements equal to it are still needed.  Uses hist[0..255].
-template <typename KeyF, typename KeepF>
+template <int NT = kFT, typename KeyF, typename KeepF>
 __device__ __noinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, uint32_t need, uint32_t *hist,
                                                   uint32_t *wtot, uint32_t *sc, uint32_t *need_left) {
     uint32_t prefix = 0, mask = 0;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += kFT) hist[i] = 0;
+        for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
         __syncthreads();
-        for (int e = threadIdx.x; e < n; e += kFT) {
+        for (int e = threadIdx.x; e < n; e += NT) {
             if (!keep(e)) continue;
             const uint32_t k = key(e);
             if (((k ^ prefix) & mask) == 0) atomicAdd(&hist[(k >> shift) & 255u], 1u);
         }
         __syncthreads();
-        cta_find_bin<1>([&](int i) { return hist[i]; }, need, wtot, sc);
+        if (NT == 256) {
+            cta_find_bin<1, NT>([&](int i) { return hist[i]; }, need, wtot, sc);
+        } else {
+            // NT threads and 256 buckets: the upper threads hold empty buckets
+            cta_find_bin<1, NT>([&](int i) { return i < 256 ? hist[i] : 0u; }, need, wtot, sc);
+        }
         prefix |= sc[0] << shift;
         mask |= 255u << shift;
         need -= sc[1];
@@ -118,15 +126,36 @@ __device__ __noinline__ uint32_t cta_radix_select(KeyF key, KeepF keep, int n, u
 }
 
 // bins[] holds one 16-bit entry per token of the chunk in token order (entry
-// p is token t0 + p).  A lane scans 8 consecutive entries with one 16-byte
-// load; these give, per 16-bit half of each word, an all-ones mask where the
-// entry's bin is above / equal to a threshold (entries hold bin + 1).
-__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return __vcmpgtu2(w & 0x3FFF3FFFu, thr2); }
-__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) { return __vcmpeq2(w & 0x3FFF3FFFu, thr2); }
-// 8-bit mask (bit j = entry j of the lane's 8) from four per-half masks
+// p is token t0 + p): bin + 1 in bits 0-13, flags in bits 14-15.  A lane
+// scans 8 consecutive entries with one 16-byte load.  The tests below give,
+// per 16-bit half of a word, a bit at position 0 (low half) or 16 (high half).
+// half_ge: [entry >= thr] for thr2 = thr * 0x10001, thr <= 0x4000.  Per half
+// v + 0x4000 - thr lies in [0, 0x7FFF] (v, thr < 0x4000 after masking the
+// flags), so the halves never borrow from each other, and its bit 14 is
+// [v >= thr].
+__device__ __forceinline__ uint32_t half_ge(uint32_t w, uint32_t thr2) {
+    return (((w & 0x3FFF3FFFu) + 0x40004000u - thr2) >> 14) & 0x00010001u;
+}
+__device__ __forceinline__ uint32_t half_gt(uint32_t w, uint32_t thr2) { return half_ge(w, thr2 + 0x10001u); }
+__device__ __forceinline__ uint32_t half_eq(uint32_t w, uint32_t thr2) {
+    return half_ge(w, thr2) & ~half_ge(w, thr2 + 0x10001u);
+}
+// The halves carrying any of the flag bits bit2 (bits 14 and / or 15 of each half).
+__device__ __forceinline__ uint32_t half_flagged(uint32_t w, uint32_t bit2) {
+    const uint32_t t = (w & bit2) >> 14;
+    return (t | (t >> 1)) & 0x00010001u;
+}
+// The flag pattern (bit 15 or 14 of each half) of the halves marked in m.
+__device__ __forceinline__ uint32_t sure_flags(uint32_t m) { return m << 15; }
+__device__ __forceinline__ uint32_t win_flags(uint32_t m) { return m << 14; }
+// 8-bit mask (bit j = entry j of the lane's 8) from the four words' half bits
 __device__ __forceinline__ uint32_t mask8(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
-    return (m0 & 1u) | ((m0 >> 15) & 2u) | ((m1 & 1u) << 2) | ((m1 >> 13) & 8u) | ((m2 & 1u) << 4) |
-           ((m2 >> 11) & 32u) | ((m3 & 1u) << 6) | ((m3 >> 9) & 128u);
+    const uint32_t a = m0 | (m1 << 2) | (m2 << 4) | (m3 << 6);   // entry 2k at bit 2k, entry 2k+1 at bit 16 + 2k
+    return (a | (a >> 15)) & 0xFFu;
+}
+// The half bits of word k (entries 2k, 2k+1) of an 8-bit per-entry mask.
+__device__ __forceinline__ uint32_t halves_of(uint32_t m8, int k) {
+    return ((m8 >> (2 * k)) & 1u) | (((m8 >> (2 * k + 1)) & 1u) << 16);
 }
 
 // Appends the tokens of bin b* (entries equal to b2 in both halves) to the
@@ -134,11 +163,12 @@ __device__ __forceinline__ uint32_t mask8(uint32_t m0, uint32_t m1, uint32_t m2,
 // by the lane that scored it (same table, same rotation, same order of
 // additions, so bit-identical).  The fallback for a CTA whose threshold bin
 // holds more tokens than the shared list takes; ties-heavy tables only.
+template <int NT = kFT>
 __device__ __noinline__ void emit_bin_tokens(const uint16_t *bins, int nrows, uint32_t b2, const float *t2,
                                              const uint4 *crow, int t0, float qmu, int *ncand, uint2 *cand, int cap) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
+    for (int row = warp; row < nrows; row += NT / 32) {
         const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
         const uint32_t eq = mask8(half_eq(w.x, b2), half_eq(w.y, b2), half_eq(w.z, b2), half_eq(w.w, b2));
         // token t0 + p was scored by lane p mod 32 (the table's bank rotation)
@@ -161,11 +191,12 @@ __device__ __noinline__ void emit_bin_tokens(const uint16_t *bins, int nrows, ui
 
 // Turns sh.rowcnt-style per-row counts into exclusive prefix sums in place and
 // returns the total.  Expects the counts to be visible; ends synchronized.
+template <int NT = kFT>
 __device__ __forceinline__ uint32_t rows_to_bases(uint32_t *rowcnt, int nrows, uint32_t *wtot) {
     uint32_t total;
     const int tid = threadIdx.x;
     const uint32_t v = tid < nrows ? rowcnt[tid] : 0u;
-    const uint32_t run = cta_excl_scan(v, wtot, &total);
+    const uint32_t run = cta_excl_scan<NT>(v, wtot, &total);
     if (tid < nrows) rowcnt[tid] = run;
     __syncthreads();
     return total;
@@ -174,28 +205,29 @@ __device__ __forceinline__ uint32_t rows_to_bases(uint32_t *rowcnt, int nrows, u
 // 8-bit mask of the entries of row `row` (8 per lane) that carry flag bit2.
 __device__ __forceinline__ uint32_t flagged8(const uint16_t *bins, int row, int lane, uint32_t bit2) {
     const uint4 w = *reinterpret_cast<const uint4 *>(bins + row * kFRow + 8 * lane);
-    return mask8(__vcmpne2(w.x & bit2, 0u), __vcmpne2(w.y & bit2, 0u), __vcmpne2(w.z & bit2, 0u),
-                 __vcmpne2(w.w & bit2, 0u));
+    return mask8(half_flagged(w.x, bit2), half_flagged(w.y, bit2), half_flagged(w.z, bit2), half_flagged(w.w, bit2));
 }
 
 // Fills list[0, wn) with the tokens of the entries flagged bit2 whose
 // ordinals (ascending token order) lie in [wbase, wbase + wn).  The fallback
 // when a pass holds more tokens than the direct list takes.  Ends synchronized.
 // (Inlined: as a call it costs the kernel spills around the call site.)
+template <int NT = kFT>
 __device__ __forceinline__ void stage_flagged(const uint16_t *bins, int nrows, uint32_t bit2, uint32_t wbase, int t0,
-                                           uint32_t *rowcnt, uint32_t *wtot, int32_t *list) {
+                                           uint32_t *rowcnt, uint32_t *wtot, int32_t *list,
+                                           uint32_t cap = kFListCap) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
+    for (int row = warp; row < nrows; row += NT / 32) {
         uint32_t cnt = __popc(flagged8(bins, row, lane, bit2));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
         if (lane == 0) rowcnt[row] = cnt;
     }
     __syncthreads();
-    rows_to_bases(rowcnt, nrows, wtot);
+    rows_to_bases<NT>(rowcnt, nrows, wtot);
 #pragma unroll 1
-    for (int row = warp; row < nrows; row += kFW) {
+    for (int row = warp; row < nrows; row += NT / 32) {
         const uint32_t m = flagged8(bins, row, lane, bit2);
         uint32_t incl = __popc(m);
 #pragma unroll
@@ -206,7 +238,7 @@ __device__ __forceinline__ void stage_flagged(const uint16_t *bins, int nrows, u
         uint32_t ord = rowcnt[row] + incl - __popc(m);
         for (uint32_t mm = m; mm; mm &= mm - 1, ++ord) {
             const int t = t0 + row * kFRow + 8 * lane + __ffs(mm) - 1;
-            if (ord >= wbase && ord < wbase + kFListCap) list[ord - wbase] = t;
+            if (ord >= wbase && ord < wbase + cap) list[ord - wbase] = t;
         }
     }
     __syncthreads();
@@ -253,6 +285,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 
 // Waits until at most one group of this thread's copies is still in flight.
 __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Waits until none of this thread's copies is in flight.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Value rows staged by a warp: two halves of its buffer, so that one half
 // is consumed while the other is in flight.
@@ -308,18 +343,40 @@ __device__ __forceinline__ void warp_fma_v(WarpSoftmax<GM> &s, const char *vb, c
 // select of the need-th key and of the lowest tied token indices, then one
 // marking pass.  Returns this thread's count of winners before the chunk.
 // Kept out of line: it only runs for heavily tied or flat score tables.
-template <typename CandF>
+template <int NT = kFT, typename CandF>
 __device__ __noinline__ uint32_t refine_by_radix(CandF cand, int ncand, uint32_t need, int t0, int chunk,
                                                  uint32_t *winbits, uint32_t *hist, uint32_t *wtot, uint32_t *sc) {
     uint32_t ties_needed, left, before = 0;
-    const uint32_t T = cta_radix_select([&](int e) { return cand(e).x; }, [&](int) { return true; }, ncand,
+    const uint32_t T = cta_radix_select<NT>([&](int e) { return cand(e).x; }, [&](int) { return true; }, ncand,
                                         need, hist, wtot, sc, &ties_needed);
     // the ties_needed lowest token indices among keys equal to T
-    const uint32_t tie_idx = ~cta_radix_select([&](int e) { return ~cand(e).y; },
+    const uint32_t tie_idx = ~cta_radix_select<NT>([&](int e) { return ~cand(e).y; },
                                                [&](int e) { return cand(e).x == T; }, ncand, ties_needed,
                                                hist, wtot, sc, &left);
-    for (int e = threadIdx.x; e < ncand; e += kFT) {
+    for (int e = threadIdx.x; e < ncand; e += NT) {
         const uint2 v = cand(e);
+        if (v.x > T || (v.x == T && v.y <= tie_idx)) {
+            const int rel = static_cast<int>(v.y) - t0;
+            if (rel >= 0 && rel < chunk) atomicOr(&winbits[rel >> 5], 1u << (rel & 31));
+            else if (rel < 0) ++before;
+        }
+    }
+    return before;
+}
+
+// The same over a candidate list in global memory.
+template <int NT = kFT>
+__device__ __noinline__ uint32_t refine_by_radix(const uint2 *cand, int ncand, uint32_t need, int t0, int chunk,
+                                                 uint32_t *winbits, uint32_t *hist, uint32_t *wtot, uint32_t *sc) {
+    uint32_t ties_needed, left, before = 0;
+    const uint32_t T = cta_radix_select<NT>([&](int e) { return __ldcg(cand + e).x; }, [&](int) { return true; }, ncand,
+                                        need, hist, wtot, sc, &ties_needed);
+    // the ties_needed lowest token indices among keys equal to T
+    const uint32_t tie_idx = ~cta_radix_select<NT>([&](int e) { return ~__ldcg(cand + e).y; },
+                                               [&](int e) { return __ldcg(cand + e).x == T; }, ncand, ties_needed,
+                                               hist, wtot, sc, &left);
+    for (int e = threadIdx.x; e < ncand; e += NT) {
+        const uint2 v = __ldcg(cand + e);
         if (v.x > T || (v.x == T && v.y <= tie_idx)) {
             const int rel = static_cast<int>(v.y) - t0;
             if (rel >= 0 && rel < chunk) atomicOr(&winbits[rel >> 5], 1u << (rel & 31));

@@ -355,10 +355,10 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
             const uint32_t gx = half_gt(w.x, b2), gy = half_gt(w.y, b2), gz = half_gt(w.z, b2), gw = half_gt(w.w, b2);
             const uint32_t ex = half_eq(w.x, b2), ey = half_eq(w.y, b2), ez = half_eq(w.z, b2), ew = half_eq(w.w, b2);
             if (gx | gy | gz | gw) {
-                w.x |= gx & kSure;
-                w.y |= gy & kSure;
-                w.z |= gz & kSure;
-                w.w |= gw & kSure;
+                w.x |= sure_flags(gx);
+                w.y |= sure_flags(gy);
+                w.z |= sure_flags(gz);
+                w.w |= sure_flags(gw);
                 *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
                 gmask |= static_cast<unsigned long long>(mask8(gx, gy, gz, gw)) << (8 * r);
             }
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                     }
                 }
             } else {
-                win_before += refine_by_radix([&](int e) { return __ldcg(cand + e); }, ncand, need, t0, a.chunk,
+                win_before += refine_by_radix(cand, ncand, need, t0, a.chunk,
                                               sh.u.sel.winbits, sh.hist, sh.wtot, sh.sc);
             }
             __syncthreads();
@@ -580,16 +580,16 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
                     const int p0 = row * kFRow + 8 * lane;
                     uint4 w = *reinterpret_cast<const uint4 *>(sh.bins + p0);
                     const uint32_t wb = (sh.u.sel.winbits[p0 >> 5] >> (p0 & 31)) & 0xFFu;
-                    // per 16-bit half: all ones where the entry is in b* and won
-                    const uint32_t hx = half_eq(w.x, b2) & (((wb & 1u) ? 0xFFFFu : 0u) | ((wb & 2u) ? 0xFFFF0000u : 0u));
-                    const uint32_t hy = half_eq(w.y, b2) & (((wb & 4u) ? 0xFFFFu : 0u) | ((wb & 8u) ? 0xFFFF0000u : 0u));
-                    const uint32_t hz = half_eq(w.z, b2) & (((wb & 16u) ? 0xFFFFu : 0u) | ((wb & 32u) ? 0xFFFF0000u : 0u));
-                    const uint32_t hw = half_eq(w.w, b2) & (((wb & 64u) ? 0xFFFFu : 0u) | ((wb & 128u) ? 0xFFFF0000u : 0u));
+                    // per 16-bit half: the entry is in b* and won
+                    const uint32_t hx = half_eq(w.x, b2) & halves_of(wb, 0);
+                    const uint32_t hy = half_eq(w.y, b2) & halves_of(wb, 1);
+                    const uint32_t hz = half_eq(w.z, b2) & halves_of(wb, 2);
+                    const uint32_t hw = half_eq(w.w, b2) & halves_of(wb, 3);
                     if (hx | hy | hz | hw) {
-                        w.x |= hx & kWin;
-                        w.y |= hy & kWin;
-                        w.z |= hz & kWin;
-                        w.w |= hw & kWin;
+                        w.x |= win_flags(hx);
+                        w.y |= win_flags(hy);
+                        w.z |= win_flags(hz);
+                        w.w |= win_flags(hw);
                         *reinterpret_cast<uint4 *>(sh.bins + p0) = w;
                     }
                 }

@@ -37,15 +37,15 @@ struct ScoreTables {
 
 constexpr int kTableThreads = 256;      // CTA size of every kernel that builds the tables
 
-// One thread's share of the inputs of the tables of segment (b, h): the
-// group's query rows (as fp32), the segment's codebook (512 float4) and its
-// channel means (128).  load() issues every global load at once; store()
+// One thread's share (of NT threads) of the inputs of the tables of segment
+// (b, h): the group's query rows (as fp32), the segment's codebook (512
+// float4) and its channel means (128).  load() issues every global load at once; store()
 // writes them to shared memory (qs: group x 128, cbs, mus), so that other
 // work can be issued in between.
-template <int DT>
+template <int DT, int NT = kTableThreads>
 struct TableInputs {
-    static constexpr int kQ = kMaxGroup * kHeadDim / kTableThreads;             // 4
-    static constexpr int kCb = kSubspaces * kClusters / kTableThreads;          // 2
+    static constexpr int kQ = kMaxGroup * kHeadDim / NT;             // 4 (256 threads) or 2 (512)
+    static constexpr int kCb = kSubspaces * kClusters / NT;          // 2 or 1
     float qv[kQ];
     float4 cv[kCb];
     float mv;
@@ -58,12 +58,12 @@ struct TableInputs {
                            (static_cast<size_t>(b) * hq + static_cast<size_t>(h) * group) * kHeadDim * EB;
 #pragma unroll
         for (int i = 0; i < kQ; ++i) {
-            const int e = tid + kTableThreads * i;
+            const int e = tid + NT * i;
             qv[i] = (e < group * kHeadDim) ? load1<DT>(qrow, e) : 0.f;
         }
         const float4 *cb = reinterpret_cast<const float4 *>(codebook) + static_cast<size_t>(seg) * kSubspaces * kClusters;
 #pragma unroll
-        for (int i = 0; i < kCb; ++i) cv[i] = __ldg(cb + tid + kTableThreads * i);
+        for (int i = 0; i < kCb; ++i) cv[i] = __ldg(cb + tid + NT * i);
         mv = (tid < kHeadDim) ? __ldg(mu + static_cast<size_t>(seg) * kHeadDim + tid) : 0.f;
     }
 
@@ -71,11 +71,11 @@ struct TableInputs {
         const int tid = threadIdx.x;
 #pragma unroll
         for (int i = 0; i < kQ; ++i) {
-            const int e = tid + kTableThreads * i;
+            const int e = tid + NT * i;
             if (e < group * kHeadDim) qs[e] = qv[i];
         }
 #pragma unroll
-        for (int i = 0; i < kCb; ++i) cbs[tid + kTableThreads * i] = cv[i];
+        for (int i = 0; i < kCb; ++i) cbs[tid + NT * i] = cv[i];
         if (tid < kHeadDim) mus[tid] = mv;
     }
 };
@@ -83,9 +83,10 @@ struct TableInputs {
 // Builds q_bar, LUT, q_bar.mu and T2 from staged inputs with the whole CTA.
 // Expects the staged inputs to be visible (a __syncthreads() after staging);
 // ends with a __syncthreads().
+template <int NT = kTableThreads>
 __device__ __forceinline__ void build_score_tables(ScoreTables &sh, const float *qs, const float4 *cbs,
                                                    const float *mus, int group) {
-    constexpr int nt = kTableThreads;
+    constexpr int nt = NT;
     const int tid = threadIdx.x;
     for (int c = tid; c < kHeadDim; c += nt) {
         float acc = qs[c];

@@ -122,6 +122,22 @@ sikv_status launch_decode_fused(const sikv_params &p, const FusedPlan &plan, con
                                 const int32_t *seq_lens, const int32_t *k_per_seq, void *out, int32_t *idx_out,
                                 float *scores_out, char *ws, int32_t *status, cudaStream_t stream);
 
+// Cluster single-launch decode (decode_cluster.cu).
+struct ClusterPlan {
+    bool ok = false;
+    int csize = 0, chunk = 0, npt = 0, gm = 0, grid = 0;
+};
+// vq: the kernel that reads 2-bit value rows for the selected tokens
+ClusterPlan cluster_plan(const sikv_params &p, bool vq = false);
+size_t fused_cand_cap(const sikv_params &p);
+// cand: the workspace candidate list ([segs][cand_cap] pairs, cand_cap >=
+// max_seq_len), used only by CTAs whose threshold bin overflows shared memory
+sikv_status launch_decode_cluster(const sikv_params &p, const ClusterPlan &plan, const void *q, const void *K,
+                                  const void *V, const uint8_t *vq, const uint8_t *codes, const float *codebook,
+                                  const float *mu, const int32_t *seq_lens, const int32_t *k_per_seq, void *out,
+                                  int32_t *idx_out, float *scores_out, uint2 *cand, size_t cand_cap, int32_t *status,
+                                  cudaStream_t stream);
+
 int device_sm_count();
 
 }  // namespace sikv

@@ -58,12 +58,12 @@ def oracle_queries(w: gen.Workload, bt: gen.Batch, step: int, b: int, h: int) ->
 class DeviceWorkload:
     """A workload uploaded to cuda:0 with its cache and workspaces."""
 
-    def __init__(self, w: gen.Workload, steps=(0,), bt: gen.Batch | None = None):
+    def __init__(self, w: gen.Workload, steps=(0,), bt: gen.Batch | None = None, decode_path: int = 0):
         dev = device()
         self.w = w
         self.bt = bt if bt is not None else gen.make_batch(w, steps)
         self.p = sk.make_params(w.dtype, w.batch, w.num_q_heads, w.num_kv_heads, w.max_seq_len, w.num_sinks,
-                                w.max_topk)
+                                w.max_topk, decode_path=decode_path)
         self.K = sk.to_device(self.bt.K, w.dtype, dev)
         self.V = sk.to_device(self.bt.V, w.dtype, dev)
         self.q = {s: sk.to_device(self.bt.q[s], w.dtype, dev) for s in self.bt.q}

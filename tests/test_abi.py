@@ -54,6 +54,10 @@ def _p(**kw):
     ({"num_sinks": -1}, False),
     ({"max_topk": -1}, False),
     ({"dtype": 7}, False),
+    ({"decode_path": 1}, True),
+    ({"decode_path": 3}, True),
+    ({"decode_path": 4}, False),
+    ({"decode_path": -1}, False),
 ])
 def test_workspace_size_validates_params(kw, ok):
     p = _p(**kw)

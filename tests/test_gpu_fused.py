@@ -1,11 +1,14 @@
-"""The single-launch decode kernel against the standalone entry points and
+"""The single-launch decode kernels against the standalone entry points and
 the oracle.
 
-sikv_decode runs one cooperative kernel whenever every CTA of the step fits on
-the device at once.  Its scores must be bit-identical to sikv_score's (same
-table, same order of additions per token), its selection identical to
-sikv_topk's on those scores, and its attention within the attention
-tolerance of sikv_sparse_attn's over that selection.
+sikv_decode runs the whole step in one launch: on thread-block clusters (one
+cluster per segment) when a segment fits 16 CTAs, else as a cooperative
+kernel when every CTA of the step fits on the device at once.  Each test
+runs both kernels (forced through sikv_params.decode_path).  Their scores must
+be bit-identical to sikv_score's (same table, same order of additions per
+token), their selection identical to sikv_topk's on those scores, and their
+attention within the attention tolerance of sikv_sparse_attn's over that
+selection.
 """
 
 import ctypes
@@ -35,6 +38,9 @@ SHAPES = {
 }
 
 
+PATHS = {"cluster": sk.SIKV_DECODE_CLUSTER, "cooperative": sk.SIKV_DECODE_COOPERATIVE}
+
+
 def _fused_runs(p):
     return int(sk.lib().sikv_decode_launches(ctypes.byref(p))) == 1
 
@@ -51,9 +57,10 @@ def _standalone(dw, step):
     return out, idx, sc
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("name", sorted(SHAPES))
-def test_fused_matches_standalone_entry_points(name):
-    dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1))
+def test_fused_matches_standalone_entry_points(name, path):
+    dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1), decode_path=PATHS[path])
     assert _fused_runs(dw.p), "the single-launch kernel should cover this shape"
     dw.encode()
     atol, rtol = gu.attn_tol(dw.w.dtype)
@@ -67,9 +74,11 @@ def test_fused_matches_standalone_entry_points(name):
         assert np.allclose(gu.to_f64(out_f), gu.to_f64(out_s), atol=atol, rtol=rtol), name
 
 
-def test_fused_repeated_calls_leave_clean_state():
-    """Every call resets the per-segment counters: repeated calls agree bit for bit."""
-    dw = gu.DeviceWorkload(SHAPES["many-chunks"](), steps=(0, 1))
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_fused_repeated_calls_leave_clean_state(path):
+    """Repeated calls agree bit for bit (the cooperative kernel resets its
+    per-segment counters; the cluster kernel keeps no state between calls)."""
+    dw = gu.DeviceWorkload(SHAPES["many-chunks"](), steps=(0, 1), decode_path=PATHS[path])
     dw.encode()
     first = [t.clone() for t in dw.decode(step=1)]
     for _ in range(3):
@@ -79,7 +88,8 @@ def test_fused_repeated_calls_leave_clean_state():
             assert torch.equal(x, y)
 
 
-def test_fused_all_scores_tied_takes_lowest_indices():
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_fused_all_scores_tied_takes_lowest_indices(path):
     """Identical keys: every score ties, the threshold bin holds every token
     (the candidate list does not fit in shared memory) and the selection falls
     back to the lowest token indices."""
@@ -93,7 +103,7 @@ def test_fused_all_scores_tied_takes_lowest_indices():
     V = gen.to_storage(rng.standard_normal((1, 1, n, 128)), "bf16")
     q = gen.to_storage(rng.standard_normal((1, 4, 128)), "bf16")
     bt = gen.Batch(w, K, V, {0: q}, np.array([n], np.int32), np.array([k], np.int32), None, {(0, 0): np.zeros(0)})
-    dw = gu.DeviceWorkload(w, bt=bt)
+    dw = gu.DeviceWorkload(w, bt=bt, decode_path=PATHS[path])
     assert _fused_runs(dw.p)
     dw.encode()
     out, idx, sc = dw.decode()
@@ -140,10 +150,13 @@ def test_decode_host_matches_device_decode(name):
         assert torch.equal(oh2, out_d.cpu()), (name, step)
 
 
-def test_batch_split_into_sub_launches_matches_oracle():
-    """More segments than one co-resident launch holds at this length: the
-    batch runs as consecutive single-launch sub-batches (here 18 + 1
-    sequences), checked against the oracle on sampled segments.  Repeated
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_batch_split_into_sub_launches_matches_oracle(path):
+    """More segments than one co-resident launch holds at this length.  The
+    cooperative kernel runs the batch as consecutive single-launch
+    sub-batches (here 18 + 1 sequences); the cluster kernel runs it as one
+    launch whose clusters do not all fit at once (later ones run in later
+    waves).  Checked against the oracle on sampled segments.  Repeated
     calls on the same workspace must give the same bytes: each sub-launch
     leaves only its own segments' coordination state zeroed, so all of them
     must share one layout (the segments sampled in sequences 1 and 2 sit
@@ -151,8 +164,8 @@ def test_batch_split_into_sub_launches_matches_oracle():
     and candidates)."""
     dev = gu.device()
     B, H, N, S, k = 19, 8, 16896, 64, 842
-    p = sk.make_params("bf16", B, H, H, N, S, k)
-    assert int(sk.lib().sikv_decode_launches(ctypes.byref(p))) == 2
+    p = sk.make_params("bf16", B, H, H, N, S, k, decode_path=PATHS[path])
+    assert int(sk.lib().sikv_decode_launches(ctypes.byref(p))) == (2 if path == "cooperative" else 1)
     g = torch.Generator().manual_seed(31)
     K = torch.randn((B, H, N, 128), generator=g).to(torch.bfloat16)
     V = torch.randn((B, H, N, 128), generator=g).to(torch.bfloat16)
