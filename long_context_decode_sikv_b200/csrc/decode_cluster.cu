@@ -7,12 +7,15 @@
 // top-k on them, dequantization fused with sparse attention over the 64 sink
 // tokens plus the selected tokens.
 //
-// Work split.  A segment is cut into C chunks (C = the cluster size, 1..16),
-// one CTA per chunk.  The per-CTA work is the cooperative kernel's
+// Work split.  A segment is cut into C chunks (C = the cluster size, 1..16)
+// of at most 32768 tokens, one CTA of 512 threads per chunk and one CTA per
+// SM (the shared memory holds a whole chunk's bins and a batch of value rows
+// for every warp).  The per-CTA work is the cooperative kernel's
 // (decode_fused.cu): build the byte table, score the chunk's code rows into
 // per-token bins and a local histogram, find the segment's threshold bin b*,
 // select the tokens above it outright and re-rank the tokens in it on exact
-// keys, attend.  The CTAs of a cluster agree through distributed shared
+// keys, attend (each pass's list split evenly over the warps, each batch's
+// value rows requested at once).  The CTAs of a cluster agree through distributed shared
 // memory and hardware cluster barriers instead of global-memory counters:
 //   #1  (prologue)  the leader (rank 0) has zeroed its segment histogram;
 //   #2  every CTA has added its counts of the bins at or above its own k-th
@@ -33,6 +36,7 @@
 // once: extra clusters simply run in later waves.
 #include <atomic>
 
+#include "cluster_common.cuh"
 #include "decode_common.cuh"
 #include "sikv_internal.h"
 
@@ -154,65 +158,6 @@ struct ClusterAttnLayout {
     static_assert(kLuth + kLuthBytes <= AxBytes<GM>::value, "staged rows and LUTs fit ax");
     static_assert(kTok + kCW * 32 * 4 <= static_cast<int>(sizeof(ScoreTables)), "batch tokens past the table");
 };
-
-// ---- cluster primitives (sm_90+ PTX) ---------------------------------------
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Every thread of every CTA of the cluster arrives (below) and later waits;
-// the wait has acquire semantics.
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
-
-// Arrival that publishes the whole CTA's earlier writes with one fence: the
-// CTA barrier orders every thread's writes before thread 0's cluster-scope
-// fence (which is cumulative), and the cluster barrier completes only after
-// thread 0 arrives behind its fence, so the matching acquire wait sees them.
-// The other threads arrive without fencing (a per-thread release would make
-// each of them wait for its own outstanding loads and prefetches).
-__device__ __forceinline__ void cluster_arrive_cta() {
-    __syncthreads();
-    if (threadIdx.x == 0) asm volatile("fence.acq_rel.cluster;" ::: "memory");
-    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-}
-
-// Arrival with no memory ordering: for the last barrier, which only keeps
-// every CTA resident until the others are done reading its shared memory.
-__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
-
-// Address of `p` (this CTA's shared memory) in the shared memory of CTA
-// `rank` of the cluster.
-__device__ __forceinline__ uint32_t dsmem_map(const void *p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                 : "=r"(r)
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ float2 dsmem_ld_f2(uint32_t addr) {
-    float2 v;
-    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void dsmem_red_add(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 
 // The threshold-bin candidates of a whole cluster, indexed 0..n-1 in rank
 // order of their CTAs: candidate e belongs to CTA r with cbase[r] <= e <

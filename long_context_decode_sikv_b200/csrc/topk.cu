@@ -4,7 +4,9 @@
 // technical summary §2.1 item 2 (top-k selection on the LUT-GEMV scores).
 // Order: score descending, then token index ascending (-0.0 == +0.0).
 //
-// One CTA of 1024 threads per segment:
+// Two kernels.  The cluster kernel (below) splits each segment's scores over
+// a thread-block cluster; the single-CTA kernel (one CTA of 1024 threads per
+// segment) serves segments longer than a cluster holds:
 //   1. min / max of the scores;
 //   2. 4096-bin histogram linear in the score over [min, max] (a monotone
 //      map, so every token in a higher bin has a strictly higher score);
@@ -17,6 +19,10 @@
 //      token order: each warp owns a contiguous run of 32-token groups
 //      (coalesced reads, ballot counts), one scan over the warps places the
 //      runs (no atomics).
+#include <atomic>
+
+#include "cluster_common.cuh"
+#include "decode_common.cuh"
 #include "sikv_common.cuh"
 #include "sikv_internal.h"
 
@@ -277,6 +283,225 @@ topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_le
     for (int i = k + tid; i < kmax; i += kTopkThreads) out[i] = -1;
 }
 
+// ---------------------------------------------------------------------------
+// Cluster top-k.  Segment s is cut into C chunks of `chunk` scores, one CTA
+// of 512 threads per chunk, the C CTAs forming one thread-block cluster.
+// Each CTA keeps its chunk's order-preserving keys in shared memory.  The k-th
+// largest key T is found digit by digit (bits 31-20, 19-8, 7-0): every CTA
+// histograms the digit of its keys that match the digits found so far and
+// adds the counts at or above its own need-th largest into the leader's
+// histogram (distributed shared memory); the leader finds the digit where the
+// running count from the top reaches the number still needed and hands it to
+// every CTA.  Then every CTA
+// counts its keys above T and equal to T, reads the other CTAs' counts, and
+// writes its selected tokens in ascending token order at its place: the
+// ties (keys equal to T) are taken lowest token first.
+// ---------------------------------------------------------------------------
+
+constexpr int kKT = 512;                  // threads per CTA (two CTAs per SM at 64 registers)
+constexpr int kKW = kKT / 32;
+constexpr int kKMaxChunk = 32768;         // keys per CTA at most
+constexpr int kKMaxCluster = 16;
+constexpr int kKDigits = 4096;            // 12-bit digits of the first two levels
+
+struct TopkClusterSmem {
+    uint32_t hist[kKDigits];              // this CTA's digit histogram
+    uint32_t mhist[kKDigits];             // leader: the cluster's
+    uint32_t wtot[kKW + 1];
+    uint32_t sc[8];
+    uint32_t bsd[2];                      // (digit, count above it), from the leader
+    uint32_t cnt[2];                      // this CTA's (keys > T, keys == T)
+    uint32_t allcnt[2 * kKMaxCluster];
+    uint32_t key[1];                      // `chunk` keys (dynamic size)
+};
+
+constexpr size_t topk_cluster_smem(int chunk) {
+    return sizeof(TopkClusterSmem) + sizeof(uint32_t) * (static_cast<size_t>(chunk) - 1);
+}
+
+__global__ void __launch_bounds__(kKT, 2)
+topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_lens,
+                    const int32_t *__restrict__ k_per_seq, int hkv, int nmax, int num_sinks, int kmax, int csize,
+                    int chunk, int32_t *__restrict__ idx, int32_t *status) {
+    extern __shared__ __align__(16) unsigned char topk_cluster_smem_raw[];
+    TopkClusterSmem &sh = *reinterpret_cast<TopkClusterSmem *>(topk_cluster_smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int C = csize;
+    const int c = static_cast<int>(cluster_ctarank());
+    const int seg = blockIdx.x / C, b = seg / hkv;
+    int32_t *out = idx + static_cast<size_t>(seg) * kmax;
+
+    // lengths (an invalid segment selects nothing but still takes part)
+    int n_tok = __ldg(seq_lens + b);
+    if (n_tok < 0 || n_tok > nmax) {
+        if (tid == 0 && c == 0) flag_error(status, SIKV_DEVERR_SEQ_LEN);
+        n_tok = 0;
+    }
+    const int n = max(n_tok - num_sinks, 0);
+    int k = __ldg(k_per_seq + b);
+    if (k < 0 || k > kmax || k > n) {
+        if (tid == 0 && c == 0) flag_error(status, SIKV_DEVERR_TOPK);
+        k = 0;
+    }
+    // this CTA's scored tokens: positions [p_lo, p_hi) of its chunk
+    const int t0 = c * chunk;
+    const int p_lo = min(max(num_sinks - t0, 0), chunk), p_hi = max(min(n_tok - t0, chunk), p_lo);
+    const float *srow = scores + static_cast<size_t>(seg) * nmax;
+    for (int p = p_lo + tid; p < p_hi; p += kKT) sh.key[p] = score_key(__ldg(srow + t0 + p));
+    for (int i = tid; i < kKDigits; i += kKT) sh.mhist[i] = 0;
+    cluster_arrive_cta();                                    // the leader's histogram is zero
+    const uint32_t mh_leader = dsmem_map(&sh.mhist[0], 0);
+
+    // the k-th key, digit by digit (bits 31-20, 19-8, 7-0)
+    uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
+#pragma unroll 1
+    for (int level = 0; level < 3; ++level) {
+        const int shift = level == 0 ? 20 : (level == 1 ? 8 : 0);
+        const uint32_t nd = level == 2 ? 256u : static_cast<uint32_t>(kKDigits);
+        for (int i = tid; i < static_cast<int>(nd); i += kKT) sh.hist[i] = 0;
+        __syncthreads();
+        if (k > 0)
+            for (int p = p_lo + tid; p < p_hi; p += kKT) {
+                const uint32_t key = sh.key[p];
+                if (((key ^ prefix) & mask) == 0) atomicAdd(&sh.hist[(key >> shift) & (nd - 1u)], 1u);
+            }
+        __syncthreads();
+        if (level == 0) cluster_wait();                      // the leader's histogram is zero
+        if (k > 0) {
+            // only the digits at or above this CTA's own need-th largest: the
+            // cluster's is never below it (0 when the CTA holds fewer keys)
+            if (tid == 0) {
+                sh.sc[2] = 0;
+                sh.sc[3] = 0;
+            }
+            __syncthreads();
+            if (level < 2)
+                cta_find_bin<kKDigits / kKT, kKT>([&](int i) { return sh.hist[i]; }, need, sh.wtot, sh.sc + 2);
+            else
+                cta_find_bin<1, kKT>([&](int i) { return i < 256 ? sh.hist[i] : 0u; }, need, sh.wtot, sh.sc + 2);
+            for (int i = static_cast<int>(sh.sc[2]) + tid; i < static_cast<int>(nd); i += kKT) {
+                const uint32_t v = sh.hist[i];
+                if (v) dsmem_red_add(mh_leader + 4u * static_cast<uint32_t>(i), v);
+            }
+        }
+        cluster_arrive_cta();                                // every count is in the leader's histogram
+        cluster_wait();
+        if (c == 0 && k > 0) {
+            if (tid == 0) {
+                sh.sc[0] = 0;
+                sh.sc[1] = 0;
+            }
+            __syncthreads();
+            if (level < 2)
+                cta_find_bin<kKDigits / kKT, kKT>([&](int i) { return sh.mhist[i]; }, need, sh.wtot, sh.sc);
+            else
+                cta_find_bin<1, kKT>([&](int i) { return i < 256 ? sh.mhist[i] : 0u; }, need, sh.wtot, sh.sc);
+            if (tid < C) {
+                dsmem_st_u32(dsmem_map(&sh.bsd[0], static_cast<uint32_t>(tid)), sh.sc[0]);
+                dsmem_st_u32(dsmem_map(&sh.bsd[1], static_cast<uint32_t>(tid)), sh.sc[1]);
+            }
+            __syncthreads();
+            for (int i = tid; i < kKDigits; i += kKT) sh.mhist[i] = 0;   // for the next level
+        }
+        cluster_arrive_cta();                                // the digit is in every CTA
+        cluster_wait();
+        if (k > 0) {
+            prefix |= sh.bsd[0] << shift;
+            mask |= (nd - 1u) << shift;
+            need -= sh.bsd[1];
+        }
+    }
+    const uint32_t T = prefix, ties_needed = need;           // the k-th key; how many keys == T are selected
+
+    // keys above T and equal to T in this CTA
+    if (tid < 2) sh.cnt[tid] = 0;
+    __syncthreads();
+    if (k > 0) {
+        uint32_t g = 0, e = 0;
+        for (int p = p_lo + tid; p < p_hi; p += kKT) {
+            const uint32_t key = sh.key[p];
+            g += key > T ? 1u : 0u;
+            e += key == T ? 1u : 0u;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, off);
+            e += __shfl_xor_sync(0xffffffffu, e, off);
+        }
+        if (lane == 0) {
+            atomicAdd(&sh.cnt[0], g);
+            atomicAdd(&sh.cnt[1], e);
+        }
+    }
+    cluster_arrive_cta();                                    // every CTA's counts are published
+    cluster_wait();
+    if (k > 0) {
+        if (tid < 2 * C) sh.allcnt[tid] = dsmem_ld_u32(dsmem_map(&sh.cnt[tid & 1], static_cast<uint32_t>(tid >> 1)));
+        __syncthreads();
+        uint32_t gt_before = 0, eq_before = 0;
+        for (int r = 0; r < c; ++r) {
+            gt_before += sh.allcnt[2 * r];
+            eq_before += sh.allcnt[2 * r + 1];
+        }
+        // this CTA's first output position, and how many of its ties are taken
+        const uint32_t base = gt_before + min(eq_before, ties_needed);
+        const uint32_t my_ties = ties_needed > eq_before ? ties_needed - eq_before : 0u;
+        // emission in ascending token order: warp w owns a contiguous run of
+        // 32-position groups; ballots count its keys above T and equal to T,
+        // one scan over the warps places the runs
+        const int len = p_hi - p_lo;
+        const int groups = (len + 31) / 32;
+        const int gpw = (groups + kKW - 1) / kKW;
+        const int q_lo = p_lo + 32 * min(warp * gpw, groups), q_hi = min(p_lo + 32 * min((warp + 1) * gpw, groups), p_hi);
+        const uint32_t below = (1u << lane) - 1u;
+        uint32_t c_gt = 0, c_eq = 0;
+        for (int q0 = q_lo; q0 < q_hi; q0 += 32) {
+            const int q = q0 + lane;
+            const uint32_t key = q < q_hi ? sh.key[q] : 0u;
+            c_gt += __popc(__ballot_sync(0xffffffffu, q < q_hi && key > T));
+            c_eq += __popc(__ballot_sync(0xffffffffu, q < q_hi && key == T));
+        }
+        if (lane == 0) {
+            sh.hist[2 * warp] = c_gt;
+            sh.hist[2 * warp + 1] = c_eq;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t g = sh.hist[2 * lane], e = sh.hist[2 * lane + 1];
+            uint32_t gi = g, ei = e;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t og = __shfl_up_sync(0xffffffffu, gi, off), oe = __shfl_up_sync(0xffffffffu, ei, off);
+                if (lane >= off) {
+                    gi += og;
+                    ei += oe;
+                }
+            }
+            sh.hist[2 * lane] = gi - g;
+            sh.hist[2 * lane + 1] = ei - e;
+        }
+        __syncthreads();
+        uint32_t tie_rank = sh.hist[2 * warp + 1];
+        uint32_t pos = base + sh.hist[2 * warp] + min(tie_rank, my_ties);
+        for (int q0 = q_lo; q0 < q_hi; q0 += 32) {
+            const int q = q0 + lane;
+            const uint32_t key = q < q_hi ? sh.key[q] : 0u;
+            const bool gt = q < q_hi && key > T, eq = q < q_hi && key == T;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool tie_sel = eq && tie_rank + __popc(eqm & below) < my_ties;
+            const uint32_t selm = __ballot_sync(0xffffffffu, gt || tie_sel);
+            if ((gt || tie_sel) && pos + __popc(selm & below) < static_cast<uint32_t>(k))
+                out[pos + __popc(selm & below)] = t0 + q;
+            pos += __popc(selm);
+            tie_rank += __popc(eqm);
+        }
+    }
+    if (c == 0)
+        for (int i = k + tid; i < kmax; i += kKT) out[i] = -1;
+    cluster_arrive_relaxed();                                // no CTA leaves while its counts are read
+    cluster_wait();
+}
+
 }  // namespace
 
 TopkLayout topk_layout(const sikv_params &) {
@@ -285,10 +510,76 @@ TopkLayout topk_layout(const sikv_params &) {
     return L;
 }
 
+namespace {
+
+// Cluster size and chunk of the cluster kernel for these parameters (0: the
+// segments are longer than a cluster holds).  The largest cluster whose whole
+// batch fits on the device at once (with a margin for how clusters pack into
+// GPCs) and whose chunks are not tiny; else the smallest cluster, whose
+// waves carry the most keys per CTA.
+int topk_cluster_plan(const sikv_params &p, int *chunk_out) {
+    const int nmax = p.max_seq_len, segs = p.batch * p.num_kv_heads;
+    const int cmin = std::max(1, (nmax + kKMaxChunk - 1) / kKMaxChunk);
+    if (cmin > kKMaxCluster) return 0;
+    const int sms = device_sm_count();
+    auto chunk_of = [&](int cs) { return ((nmax + cs - 1) / cs + 31) / 32 * 32; };
+    int csize = cmin;
+    for (int cs = kKMaxCluster; cs > std::max(cmin, 1); --cs) {
+        const int ch = chunk_of(cs);
+        if (ch < 2048 || (nmax + ch - 1) / ch != cs) continue;
+        // CTAs per SM: two by registers (64 per thread), fewer when the keys need more shared memory
+        const int bps = std::min<int>(2, static_cast<int>(233472 / (topk_cluster_smem(ch) + 1024)));
+        if (10 * segs * cs <= 9 * sms * bps) {
+            csize = cs;
+            break;
+        }
+    }
+    *chunk_out = chunk_of(csize);
+    // one CTA per segment: the single-CTA kernel (1024 threads) does that better
+    if (csize == 1) return 0;
+    return *chunk_out <= kKMaxChunk ? csize : 0;
+}
+
+}  // namespace
+
 sikv_status launch_topk(const sikv_params &p, const float *scores, const int32_t *seq_lens,
                         const int32_t *k_per_seq, int32_t *idx, int32_t *status,
                         cudaStream_t stream) {
+    // per device: 0 unknown, 1 the cluster kernel launches, 2 it does not
+    // (then the single-CTA kernel serves every call)
+    static std::atomic<int> usable[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
     const int segs = p.batch * p.num_kv_heads;
+    int chunk = 0;
+    const int csize = (dev >= 0 && usable[dev].load(std::memory_order_relaxed) != 2) ? topk_cluster_plan(p, &chunk) : 0;
+    if (csize > 0) {
+        const size_t smem = topk_cluster_smem(chunk);
+        if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(topk_cluster_smem(kKMaxChunk))) == cudaSuccess &&
+            cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(segs * csize));
+            cfg.blockDim = dim3(kKT);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = static_cast<unsigned>(csize);
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, seq_lens, k_per_seq, p.num_kv_heads,
+                                   p.max_seq_len, p.num_sinks, p.max_topk, csize, chunk, idx, status) == cudaSuccess) {
+                usable[dev].store(1, std::memory_order_relaxed);
+                return SIKV_OK;
+            }
+        }
+        cudaGetLastError();                  // a configuration the device refuses: the single-CTA kernel
+        usable[dev].store(2, std::memory_order_relaxed);
+    }
     const size_t smem = sizeof(TopkSmem);
     if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SIKV_ERR_CUDA;
