@@ -180,6 +180,9 @@ SIKV_API int32_t sikv_decode_resolved_path(const sikv_params *p);
  *                 K[t][4s:4s+4] - mu[4s:4s+4]; 0 for an empty cluster;
  *   counts      = cluster sizes (optional output, may be NULL).
  * Inputs: K (dtype), seq_lens.  Outputs: mu, codes, codebook, counts.
+ * The workspace holds per-chunk partial sums.  Its size depends on the
+ * current device: the chunk length is chosen so that the chunk CTAs fill
+ * whole waves of its SMs, so query the size on the device that runs the call.
  */
 SIKV_API sikv_status sikv_encode_keys(const sikv_params *p, const void *K, const int32_t *seq_lens,
                              float *mu, uint8_t *codes, float *codebook, int32_t *counts,

@@ -255,7 +255,7 @@ sikv_status sikv_check_device_status(void *workspace, size_t workspace_bytes, si
 
 size_t sikv_encode_workspace_size(const sikv_params *p) {
     if (check_params(p) != SIKV_OK) return 0;
-    return encode_layout(*p).total;
+    return encode_layout(*p, device_sm_count()).total;
 }
 
 size_t sikv_score_workspace_size(const sikv_params *p) {
@@ -387,8 +387,9 @@ sikv_status sikv_encode_keys(const sikv_params *p, const void *K, const int32_t 
     SIKV_REQUIRE_PTR(codes);
     SIKV_REQUIRE_PTR(codebook);
     if (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)) return SIKV_ERR_UNSUPPORTED;
-    SIKV_TRY(check_ws(workspace, workspace_bytes, encode_layout(*p).total));
-    return launch_encode(*p, K, seq_lens, mu, codes, codebook, counts, static_cast<char *>(workspace),
+    const EncodeLayout L = encode_layout(*p, device_sm_count());
+    SIKV_TRY(check_ws(workspace, workspace_bytes, L.total));
+    return launch_encode(*p, L, K, seq_lens, mu, codes, codebook, counts, static_cast<char *>(workspace),
                          reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -41,13 +41,13 @@ struct DecodeLayout {
     size_t total = 0;
 };
 
-EncodeLayout encode_layout(const sikv_params &p);
+EncodeLayout encode_layout(const sikv_params &p, int num_sms);
 TopkLayout topk_layout(const sikv_params &p);
 AttnLayout attn_layout(const sikv_params &p, size_t base);
 DecodeLayout decode_layout(const sikv_params &p);
 
-sikv_status launch_encode(const sikv_params &p, const void *K, const int32_t *seq_lens, float *mu,
-                          uint8_t *codes, float *codebook, int32_t *counts, char *ws,
+sikv_status launch_encode(const sikv_params &p, const EncodeLayout &L, const void *K, const int32_t *seq_lens,
+                          float *mu, uint8_t *codes, float *codebook, int32_t *counts, char *ws,
                           cudaStream_t stream);
 
 // Dense comparison baselines (dense.cu).

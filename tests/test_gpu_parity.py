@@ -69,6 +69,45 @@ def test_encode_bit_exact(name):
             assert np.allclose(cb[b, h], o.cent, rtol=1e-5, atol=1e-6 * scale), (b, h)
 
 
+def test_encode_mean_exact_outside_the_fast_window():
+    """bf16 keys with values the encoder's plain fp64 channel sums cannot take
+    exactly (zeros of both signs, subnormals, values just outside
+    [2^-20, 2^17), very small and very large values) among ordinary ones, a
+    head whose every value is tiny, and a head of values at the window's two
+    edges only: the channel mean stays bit-exact, the codes and cluster sizes
+    exact."""
+    w = gen.small(1, n=4096 + 700, batch=1, num_q_heads=12, num_kv_heads=3)
+    bt = gen.make_batch(w, steps=(0,))
+    n = w.seq_lens[0]
+    rng = np.random.default_rng(np.random.SeedSequence([4096, 700, 3]))
+    K = gen.storage_to_f64(bt.K, w.dtype).astype(np.float32)
+    special = np.array([0.0, -0.0, 2.0 ** -130, -(2.0 ** -133), 2.0 ** -21, -(2.0 ** -21), 2.0 ** -20,
+                        -(2.0 ** -20), 2.0 ** 17, -(2.0 ** 17), 130560.0, -130560.0, 1e-30, -1e-30, 1e20,
+                        -3e19], np.float32)
+    h0 = K[0, 0, :n]
+    hit = rng.random(h0.shape) < 2e-4
+    h0[hit] = rng.choice(special, size=int(hit.sum()))
+    K[0, 1, :n] *= np.float32(2.0 ** -30)
+    edge = np.where(rng.random((n, 128)) < 0.5, np.float32(2.0 ** -20), np.float32(130560.0))
+    K[0, 2, :n] = edge * rng.choice(np.array([-1.0, 1.0], np.float32), size=(n, 128))
+    bt.K = gen.to_storage(K, w.dtype)
+    dw = gu.DeviceWorkload(w, steps=(0,), bt=bt)
+    dw.encode()
+    mu = dw.cache.mu.cpu().numpy()
+    codes = dw.cache.codes.cpu().numpy()
+    counts = dw.cache.counts.cpu().numpy()
+    cb = dw.cache.codebook.cpu().numpy()
+    for h in range(w.num_kv_heads):
+        o = gu.oracle_head(w, bt, 0, h)
+        assert np.array_equal(mu[0, h].view(np.uint32), o.mu.view(np.uint32)), h
+        assert np.array_equal(codes[0, h, :n], oracle.pack_codes(o.code)), h
+        assert np.array_equal(counts[0, h], o.counts), h
+        scale = max(1.0, float(np.abs(o.cent).max()))
+        assert np.allclose(cb[0, h], o.cent, rtol=1e-5, atol=1e-6 * scale), h
+    del dw
+    torch.cuda.empty_cache()
+
+
 def _upload_oracle_encode(dw):
     """Oracle encode outputs (mu, packed codes, fp32 centroids) as device tensors."""
     w, dev = dw.w, dw.dev
