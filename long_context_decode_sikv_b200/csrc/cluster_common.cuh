@@ -66,6 +66,12 @@ __device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void dsmem_red_add(uint32_t addr, uint32_t v) {
     asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+// Adds v to the word at a cluster shared-memory address; returns its old value.
+__device__ __forceinline__ uint32_t dsmem_atom_add(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
+}
 
 }  // namespace
 

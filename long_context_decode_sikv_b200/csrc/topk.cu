@@ -303,15 +303,19 @@ constexpr int kKW = kKT / 32;
 constexpr int kKMaxChunk = 32768;         // keys per CTA at most
 constexpr int kKMaxCluster = 16;
 constexpr int kKDigits = 4096;            // 12-bit digits of the first two levels
+constexpr uint32_t kKCandCap = kKDigits;  // threshold-digit keys the leader can take (its mhist)
+static_assert(2 * (kKT / 32) <= kKDigits, "the warps' emission counts fit mhist");
 
 struct TopkClusterSmem {
     uint32_t hist[kKDigits];              // this CTA's digit histogram
     uint32_t mhist[kKDigits];             // leader: the cluster's
     uint32_t wtot[kKW + 1];
     uint32_t sc[8];
-    uint32_t bsd[2];                      // (digit, count above it), from the leader
+    uint32_t bsd[3];                      // (digit, count above it, keys in it), from the leader
+    uint32_t ccount;                      // leader: threshold-digit keys gathered so far
     uint32_t cnt[2];                      // this CTA's (keys > T, keys == T)
     uint32_t allcnt[2 * kKMaxCluster];
+    uint32_t gmask[2 * (kKMaxChunk / 32)];// per 32-key group: keys above T, keys equal to T
     uint32_t key[1];                      // `chunk` keys (dynamic size)
 };
 
@@ -347,13 +351,30 @@ topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict_
     const int t0 = c * chunk;
     const int p_lo = min(max(num_sinks - t0, 0), chunk), p_hi = max(min(n_tok - t0, chunk), p_lo);
     const float *srow = scores + static_cast<size_t>(seg) * nmax;
-    for (int p = p_lo + tid; p < p_hi; p += kKT) sh.key[p] = score_key(__ldg(srow + t0 + p));
+    // emission layout: warp w owns 32-key groups [g_lo, g_hi) of [p_lo, p_hi)
+    const int groups = (p_hi - p_lo + 31) / 32;
+    const int gpw = (groups + kKW - 1) / kKW;
+    const int g_lo = min(warp * gpw, groups), g_hi = min((warp + 1) * gpw, groups);
+    {
+        // eight independent loads in flight per thread
+        int p = p_lo + tid;
+        for (; p + 7 * kKT < p_hi; p += 8 * kKT) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(srow + t0 + p + u * kKT);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sh.key[p + u * kKT] = score_key(v[u]);
+        }
+        for (; p < p_hi; p += kKT) sh.key[p] = score_key(__ldg(srow + t0 + p));
+    }
     for (int i = tid; i < kKDigits; i += kKT) sh.mhist[i] = 0;
+    if (tid == 0) sh.ccount = 0;
     cluster_arrive_cta();                                    // the leader's histogram is zero
     const uint32_t mh_leader = dsmem_map(&sh.mhist[0], 0);
 
     // the k-th key, digit by digit (bits 31-20, 19-8, 7-0)
     uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
+    bool fast = false;
 #pragma unroll 1
     for (int level = 0; level < 3; ++level) {
         const int shift = level == 0 ? 20 : (level == 1 ? 8 : 0);
@@ -399,6 +420,7 @@ topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict_
             if (tid < C) {
                 dsmem_st_u32(dsmem_map(&sh.bsd[0], static_cast<uint32_t>(tid)), sh.sc[0]);
                 dsmem_st_u32(dsmem_map(&sh.bsd[1], static_cast<uint32_t>(tid)), sh.sc[1]);
+                dsmem_st_u32(dsmem_map(&sh.bsd[2], static_cast<uint32_t>(tid)), sh.mhist[sh.sc[0]]);
             }
             __syncthreads();
             for (int i = tid; i < kKDigits; i += kKT) sh.mhist[i] = 0;   // for the next level
@@ -410,27 +432,132 @@ topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict_
             mask |= (nd - 1u) << shift;
             need -= sh.bsd[1];
         }
+        // few keys share the first digit of the k-th: the leader finishes alone
+        if (level == 0 && k > 0 && sh.bsd[2] <= kKCandCap) {
+            fast = true;
+            break;
+        }
+    }
+    if (fast) {
+        // every key of the threshold digit into the leader's mhist (it holds
+        // bsd[2] <= kKCandCap of them): gathered in this CTA's hist first, then
+        // one range of the leader's list reserved for the CTA
+        // This CTA's candidates are its level-0 count of the threshold digit:
+        // their range of the leader's list is reserved before the scan, which
+        // hides the round trip.
+        const uint32_t below = (1u << lane) - 1u;
+        uint32_t at0 = 0;
+        if (tid == 0) {
+            const uint32_t mine = min(sh.hist[prefix >> 20], kKCandCap);
+            at0 = mine ? dsmem_atom_add(dsmem_map(&sh.ccount, 0), mine) : 0u;
+            sh.cnt[0] = 0;
+        }
+        __syncthreads();
+        for (int base = p_lo; base < p_hi; base += kKT) {
+            const int p = base + tid;
+            const uint32_t key = p < p_hi ? sh.key[p] : 0u;
+            const bool cand = p < p_hi && ((key ^ prefix) & mask) == 0;
+            const uint32_t m = __ballot_sync(0xffffffffu, cand);
+            if (m) {
+                uint32_t slot = 0;
+                if (lane == 0) slot = atomicAdd(&sh.cnt[0], static_cast<uint32_t>(__popc(m)));
+                slot = __shfl_sync(0xffffffffu, slot, 0) + static_cast<uint32_t>(__popc(m & below));
+                if (cand && slot < kKCandCap) sh.hist[slot] = key;
+            }
+        }
+        __syncthreads();
+        const uint32_t nmine = min(sh.cnt[0], kKCandCap);
+        if (tid == 0) sh.sc[4] = at0;
+        __syncthreads();
+        {
+            const uint32_t cbuf = dsmem_map(&sh.mhist[0], 0), at = sh.sc[4];
+            for (uint32_t i = tid; i < nmine; i += kKT)
+                if (at + i < kKCandCap) dsmem_st_u32(cbuf + 4u * (at + i), sh.hist[i]);
+        }
+        cluster_arrive_cta();                                // the leader holds every candidate
+        cluster_wait();
+        if (c == 0) {
+            // the need-th largest candidate: bits 19-10, then bits 9-0
+            constexpr uint32_t kSub = 1024;
+            const int nc = static_cast<int>(min(sh.ccount, kKCandCap));
+            for (int i = tid; i < static_cast<int>(kSub); i += kKT) sh.hist[i] = 0;
+            if (tid == 0) {
+                sh.sc[0] = 0;
+                sh.sc[1] = 0;
+            }
+            __syncthreads();
+            for (int i = tid; i < nc; i += kKT) atomicAdd(&sh.hist[(sh.mhist[i] >> 10) & (kSub - 1u)], 1u);
+            __syncthreads();
+            cta_find_bin<kSub / kKT, kKT>([&](int i) { return sh.hist[i]; }, need, sh.wtot, sh.sc);
+            const uint32_t d1 = sh.sc[0], above1 = sh.sc[1];
+            for (int i = tid; i < static_cast<int>(kSub); i += kKT) sh.hist[i] = 0;
+            if (tid == 0) {
+                sh.sc[0] = 0;
+                sh.sc[1] = 0;
+            }
+            __syncthreads();
+            for (int i = tid; i < nc; i += kKT) {
+                const uint32_t key = sh.mhist[i];
+                if (((key >> 10) & (kSub - 1u)) == d1) atomicAdd(&sh.hist[key & (kSub - 1u)], 1u);
+            }
+            __syncthreads();
+            cta_find_bin<kSub / kKT, kKT>([&](int i) { return sh.hist[i]; }, need - above1, sh.wtot, sh.sc);
+            if (tid < C) {
+                dsmem_st_u32(dsmem_map(&sh.bsd[0], static_cast<uint32_t>(tid)), prefix | (d1 << 10) | sh.sc[0]);
+                dsmem_st_u32(dsmem_map(&sh.bsd[1], static_cast<uint32_t>(tid)), need - above1 - sh.sc[1]);
+            }
+        }
+        cluster_arrive_cta();                                // the k-th key is in every CTA
+        cluster_wait();
+        prefix = sh.bsd[0];
+        need = sh.bsd[1];
     }
     const uint32_t T = prefix, ties_needed = need;           // the k-th key; how many keys == T are selected
 
-    // keys above T and equal to T in this CTA
-    if (tid < 2) sh.cnt[tid] = 0;
-    __syncthreads();
+    // Keys above T and equal to T, in ascending token order: warp w owns a
+    // contiguous run of 32-position groups; one ballot pass records each
+    // group's two masks (above at gmask[2 g], equal at gmask[2 g + 1]) and the
+    // warp's counts (in mhist[2 w], mhist[2 w + 1]); the CTA's totals go to
+    // the cluster; then the selections are written from the masks.
     if (k > 0) {
-        uint32_t g = 0, e = 0;
-        for (int p = p_lo + tid; p < p_hi; p += kKT) {
-            const uint32_t key = sh.key[p];
-            g += key > T ? 1u : 0u;
-            e += key == T ? 1u : 0u;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, off);
-            e += __shfl_xor_sync(0xffffffffu, e, off);
+        uint32_t c_gt = 0, c_eq = 0;
+        for (int g = g_lo; g < g_hi; ++g) {
+            const int q = p_lo + 32 * g + lane;
+            const uint32_t key = q < p_hi ? sh.key[q] : 0u;
+            const uint32_t gm = __ballot_sync(0xffffffffu, q < p_hi && key > T);
+            const uint32_t em = __ballot_sync(0xffffffffu, q < p_hi && key == T);
+            if (lane == 0) {
+                sh.gmask[2 * g] = gm;
+                sh.gmask[2 * g + 1] = em;
+            }
+            c_gt += __popc(gm);
+            c_eq += __popc(em);
         }
         if (lane == 0) {
-            atomicAdd(&sh.cnt[0], g);
-            atomicAdd(&sh.cnt[1], e);
+            sh.mhist[2 * warp] = c_gt;
+            sh.mhist[2 * warp + 1] = c_eq;
+        }
+    }
+    __syncthreads();
+    if (k > 0 && warp == 0) {
+        // exclusive scans of the warps' counts; lane 0 also writes the totals
+        const uint32_t g = lane < kKW ? sh.mhist[2 * lane] : 0u, e = lane < kKW ? sh.mhist[2 * lane + 1] : 0u;
+        uint32_t gi = g, ei = e;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t og = __shfl_up_sync(0xffffffffu, gi, off), oe = __shfl_up_sync(0xffffffffu, ei, off);
+            if (lane >= off) {
+                gi += og;
+                ei += oe;
+            }
+        }
+        if (lane < kKW) {
+            sh.mhist[2 * lane] = gi - g;
+            sh.mhist[2 * lane + 1] = ei - e;
+        }
+        if (lane == 31) {
+            sh.cnt[0] = gi;
+            sh.cnt[1] = ei;
         }
     }
     cluster_arrive_cta();                                    // every CTA's counts are published
@@ -446,54 +573,21 @@ topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict_
         // this CTA's first output position, and how many of its ties are taken
         const uint32_t base = gt_before + min(eq_before, ties_needed);
         const uint32_t my_ties = ties_needed > eq_before ? ties_needed - eq_before : 0u;
-        // emission in ascending token order: warp w owns a contiguous run of
-        // 32-position groups; ballots count its keys above T and equal to T,
-        // one scan over the warps places the runs
-        const int len = p_hi - p_lo;
-        const int groups = (len + 31) / 32;
-        const int gpw = (groups + kKW - 1) / kKW;
-        const int q_lo = p_lo + 32 * min(warp * gpw, groups), q_hi = min(p_lo + 32 * min((warp + 1) * gpw, groups), p_hi);
         const uint32_t below = (1u << lane) - 1u;
-        uint32_t c_gt = 0, c_eq = 0;
-        for (int q0 = q_lo; q0 < q_hi; q0 += 32) {
-            const int q = q0 + lane;
-            const uint32_t key = q < q_hi ? sh.key[q] : 0u;
-            c_gt += __popc(__ballot_sync(0xffffffffu, q < q_hi && key > T));
-            c_eq += __popc(__ballot_sync(0xffffffffu, q < q_hi && key == T));
-        }
-        if (lane == 0) {
-            sh.hist[2 * warp] = c_gt;
-            sh.hist[2 * warp + 1] = c_eq;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const uint32_t g = sh.hist[2 * lane], e = sh.hist[2 * lane + 1];
-            uint32_t gi = g, ei = e;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t og = __shfl_up_sync(0xffffffffu, gi, off), oe = __shfl_up_sync(0xffffffffu, ei, off);
-                if (lane >= off) {
-                    gi += og;
-                    ei += oe;
-                }
+        uint32_t tie_rank = sh.mhist[2 * warp + 1];
+        uint32_t pos = base + sh.mhist[2 * warp] + min(tie_rank, my_ties);
+        for (int g = g_lo; g < g_hi; ++g) {
+            const uint32_t gm = sh.gmask[2 * g], em = sh.gmask[2 * g + 1];
+            if ((gm | em) == 0u) continue;
+            // ties are taken while this CTA's share lasts, lowest positions first
+            const bool tie_sel = ((em >> lane) & 1u) && tie_rank + static_cast<uint32_t>(__popc(em & below)) < my_ties;
+            const uint32_t selm = gm | __ballot_sync(0xffffffffu, tie_sel);
+            if ((selm >> lane) & 1u) {
+                const uint32_t at = pos + static_cast<uint32_t>(__popc(selm & below));
+                if (at < static_cast<uint32_t>(k)) out[at] = t0 + p_lo + 32 * g + lane;
             }
-            sh.hist[2 * lane] = gi - g;
-            sh.hist[2 * lane + 1] = ei - e;
-        }
-        __syncthreads();
-        uint32_t tie_rank = sh.hist[2 * warp + 1];
-        uint32_t pos = base + sh.hist[2 * warp] + min(tie_rank, my_ties);
-        for (int q0 = q_lo; q0 < q_hi; q0 += 32) {
-            const int q = q0 + lane;
-            const uint32_t key = q < q_hi ? sh.key[q] : 0u;
-            const bool gt = q < q_hi && key > T, eq = q < q_hi && key == T;
-            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-            const bool tie_sel = eq && tie_rank + __popc(eqm & below) < my_ties;
-            const uint32_t selm = __ballot_sync(0xffffffffu, gt || tie_sel);
-            if ((gt || tie_sel) && pos + __popc(selm & below) < static_cast<uint32_t>(k))
-                out[pos + __popc(selm & below)] = t0 + q;
-            pos += __popc(selm);
-            tie_rank += __popc(eqm);
+            pos += static_cast<uint32_t>(__popc(selm));
+            tie_rank += static_cast<uint32_t>(__popc(em));
         }
     }
     if (c == 0)
