@@ -265,11 +265,12 @@ SIKV_API sikv_status sikv_decode(const sikv_params *p, const void *q, const void
 
 /*
  * sikv_decode_host -- sikv_decode with the query and the output in host
- * memory: q_host and out_host are [B][Hq][D] in the cache dtype.  Page-locked
- * buffers (cudaHostAlloc, cudaHostRegister) are device-addressable, so the
- * decode kernels read the query and write the output in place over the host
- * link; pageable buffers are staged through the workspace with
- * cudaMemcpyAsync (then the copies synchronize with the host).  Everything is
+ * memory: q_host and out_host are [B][Hq][D] in the cache dtype.  The query
+ * is staged in the workspace: from a page-locked buffer (cudaHostAlloc,
+ * cudaHostRegister; device-addressable) by a copy kernel that reads it once
+ * over the host link, otherwise by cudaMemcpyAsync.  A page-locked output
+ * buffer is written in place by the decode kernels; a pageable one is staged
+ * through the workspace (pageable copies synchronize with the host).  Everything is
  * enqueued on `stream`; returns once enqueued, and out_host is valid after
  * the stream is synchronized.  K,
  * V, codes, codebook, mu, seq_lens and k_per_seq are device pointers as for

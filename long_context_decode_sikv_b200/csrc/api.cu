@@ -130,6 +130,12 @@ HostLayout host_layout(const sikv_params &p, size_t decode_total) {
 
 // The device address of a page-locked host buffer, or null for pageable
 // memory (which then goes through a staged copy).
+// Copies n16 16-byte words from host-mapped memory into device memory: each
+// word crosses the host link once, and a warp reads 512 contiguous bytes.
+__global__ void __launch_bounds__(256) upload16_kernel(const uint4 *src, uint4 *__restrict__ dst, int n16) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += gridDim.x * blockDim.x) dst[i] = src[i];
+}
+
 void *device_view(const void *host) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
@@ -519,15 +525,23 @@ sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const voi
     SIKV_TRY(check_ws(workspace, workspace_bytes, H.total));
     char *ws = static_cast<char *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // page-locked host buffers are device-addressable (unified addressing):
-    // the kernels then read the query and write the output in place, over the
-    // host link, with no staging copy; pageable buffers are staged in the
-    // workspace with cudaMemcpyAsync
-    const void *q_dev = sikv::device_view(q_host);
+    // Page-locked host buffers are device-addressable (unified addressing).
+    // The query is read by every CTA of its segment, so it is brought into the
+    // workspace first: by a copy kernel that reads each byte of the host
+    // buffer once (a 32 KB DMA copy costs more, in latency), or, for pageable
+    // or unaligned buffers, by cudaMemcpyAsync.  The output, written once, goes
+    // to a page-locked buffer in place.
+    const void *q_view = sikv::device_view(q_host);
     void *out_dev = sikv::device_view(out_host);
-    if (!q_dev) {
-        if (cudaMemcpyAsync(ws + H.q, q_host, H.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return SIKV_ERR_CUDA;
-        q_dev = ws + H.q;
+    if (out_dev && (reinterpret_cast<uintptr_t>(out_dev) & 15u) != 0) out_dev = nullptr;   // kernels store in pairs
+    char *q_dev = ws + H.q;
+    if (q_view && (reinterpret_cast<uintptr_t>(q_view) & 15u) == 0 && H.bytes % 16 == 0) {
+        const int n16 = static_cast<int>(H.bytes / 16);
+        sikv::upload16_kernel<<<std::min((n16 + 255) / 256, 64), 256, 0, s>>>(
+            static_cast<const uint4 *>(q_view), reinterpret_cast<uint4 *>(q_dev), n16);
+        if (cudaGetLastError() != cudaSuccess) return SIKV_ERR_CUDA;
+    } else if (cudaMemcpyAsync(q_dev, q_host, H.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        return SIKV_ERR_CUDA;
     }
     SIKV_TRY(sikv::decode_step(*p, q_dev, K, V, nullptr, codes, codebook, mu, seq_lens, k_per_seq,
                                out_dev ? out_dev : ws + H.out, nullptr, nullptr, workspace, decode_total, s));
