@@ -533,7 +533,6 @@ sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const voi
     // to a page-locked buffer in place.
     const void *q_view = sikv::device_view(q_host);
     void *out_dev = sikv::device_view(out_host);
-    if (out_dev && (reinterpret_cast<uintptr_t>(out_dev) & 15u) != 0) out_dev = nullptr;   // kernels store in pairs
     char *q_dev = ws + H.q;
     if (q_view && (reinterpret_cast<uintptr_t>(q_view) & 15u) == 0 && H.bytes % 16 == 0) {
         const int n16 = static_cast<int>(H.bytes / 16);

@@ -882,27 +882,19 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(ClusterArgs a) {
             for (int r = 0; r < C; ++r) wts[r * GM + tid] *= inv;
         }
         __syncthreads();
-        // channel pairs (d, d + 1): one 4- or 8-byte store each (the output
-        // may be host memory, where narrow stores are costly)
-        const int npr = group * kHeadDim / 2;
-        const int per = (npr + C - 1) / C;
-        const int e1 = min((c + 1) * per, npr);
+        const int nel = group * kHeadDim;
+        const int per = (nel + C - 1) / C;
+        const int e1 = min((c + 1) * per, nel);
         for (int e = c * per + tid; e < e1; e += kCT) {
-            const int g = e / (kHeadDim / 2), d = 2 * (e % (kHeadDim / 2));
+            const int g = e / kHeadDim, d = e % kHeadDim;
             const uint32_t off = 4u * static_cast<uint32_t>(g * kHeadDim + d);
-            float2 acc = make_float2(0.f, 0.f);
-            for (int r = 0; r < C; ++r) {
-                const float w = wts[r * GM + g];
-                const float2 v = dsmem_ld_f2(sh.rbase[r] + off);
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-            }
+            float acc = 0.f;
+            for (int r = 0; r < C; ++r) acc = fmaf(wts[r * GM + g], dsmem_ld_f32(sh.rbase[r] + off), acc);
             const size_t orow = (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group + g) * kHeadDim + d;
             if (DT == SIKV_DTYPE_F32)
-                *reinterpret_cast<float2 *>(static_cast<float *>(a.out) + orow) = acc;
+                static_cast<float *>(a.out)[orow] = acc;
             else
-                *reinterpret_cast<uint32_t *>(static_cast<unsigned short *>(a.out) + orow) =
-                    f32_to_bf16_bits(acc.x) | (f32_to_bf16_bits(acc.y) << 16);
+                static_cast<unsigned short *>(a.out)[orow] = static_cast<unsigned short>(f32_to_bf16_bits(acc));
         }
     }
     if (a.idx_out && c == 0) {

@@ -751,23 +751,18 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
     if (!sh.last) return;
     __threadfence();
     {
-        // this thread's output pairs (d, d + 1) of head g, e = tid + kFT i with
-        // g = e / 64, d = 2 (e % 64): one 4- or 8-byte store per pair (the
-        // output may be host memory, where narrow stores are costly); the
-        // first kFPre partials of each are fetched together with the (m, l)
-        // pairs
-        constexpr int kPr = GM * kHeadDim / 2 / kFT;   // 1 or 2
-        constexpr int kFPre = kPr == 1 ? 16 : 8;
+        // this thread's output elements e = tid + kFT i; the first kFPre
+        // partials of each are fetched together with the (m, l) pairs
+        constexpr int kEl = GM * kHeadDim / kFT;       // 2 or 4
+        constexpr int kFPre = kEl == 2 ? 16 : 8;
         const size_t seg_p = static_cast<size_t>(seg) * a.cps;
-        float2 pre[kPr][kFPre];
+        float pre[kEl][kFPre];
 #pragma unroll
-        for (int i = 0; i < kPr; ++i) {
-            const int e = tid + kFT * i, g = e / (kHeadDim / 2), d = 2 * (e % (kHeadDim / 2));
+        for (int i = 0; i < kEl; ++i) {
+            const int e = tid + kFT * i, g = e / kHeadDim, d = e % kHeadDim;
 #pragma unroll
             for (int cc = 0; cc < kFPre; ++cc)
-                pre[i][cc] = (g < group && cc < a.cps)
-                                 ? __ldcg(reinterpret_cast<const float2 *>(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d))
-                                 : make_float2(0.f, 0.f);
+                pre[i][cc] = (g < group && cc < a.cps) ? __ldcg(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d) : 0.f;
         }
         float2 *mls = reinterpret_cast<float2 *>(&sh.u.at.red[0][0][0]);       // [cps][GM]
         float *wts = reinterpret_cast<float *>(mls + kFusedMaxCps * GM);       // [cps][GM]
@@ -788,30 +783,20 @@ __global__ void __launch_bounds__(kFT, 2) decode_fused_kernel(FusedArgs a) {
         }
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < kPr; ++i) {
-            const int e = tid + kFT * i, g = e / (kHeadDim / 2), d = 2 * (e % (kHeadDim / 2));
+        for (int i = 0; i < kEl; ++i) {
+            const int e = tid + kFT * i, g = e / kHeadDim, d = e % kHeadDim;
             if (g >= group) continue;
-            float2 acc = make_float2(0.f, 0.f);
+            float acc = 0.f;
 #pragma unroll
-            for (int cc = 0; cc < kFPre; ++cc) {
-                const float w = wts[min(cc, a.cps - 1) * GM + g];
-                acc.x = fmaf(w, pre[i][cc].x, acc.x);
-                acc.y = fmaf(w, pre[i][cc].y, acc.y);
-            }
+            for (int cc = 0; cc < kFPre; ++cc) acc = fmaf(wts[min(cc, a.cps - 1) * GM + g], pre[i][cc], acc);
 #pragma unroll 4
-            for (int cc = kFPre; cc < a.cps; ++cc) {
-                const float w = wts[cc * GM + g];
-                const float2 v =
-                    __ldcg(reinterpret_cast<const float2 *>(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d));
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-            }
+            for (int cc = kFPre; cc < a.cps; ++cc)
+                acc = fmaf(wts[cc * GM + g], __ldcg(a.part_o + ((seg_p + cc) * GM + g) * kHeadDim + d), acc);
             const size_t orow = (static_cast<size_t>(b) * a.hq + static_cast<size_t>(h) * group + g) * kHeadDim + d;
             if (DT == SIKV_DTYPE_F32)
-                *reinterpret_cast<float2 *>(static_cast<float *>(a.out) + orow) = acc;
+                static_cast<float *>(a.out)[orow] = acc;
             else
-                *reinterpret_cast<uint32_t *>(static_cast<unsigned short *>(a.out) + orow) =
-                    f32_to_bf16_bits(acc.x) | (f32_to_bf16_bits(acc.y) << 16);
+                static_cast<unsigned short *>(a.out)[orow] = static_cast<unsigned short>(f32_to_bf16_bits(acc));
         }
     }
     if (a.idx_out) {

@@ -119,9 +119,10 @@ def test_fused_all_scores_tied_takes_lowest_indices(path):
 
 @pytest.mark.parametrize("name", ["gqa5", "ragged-empty-chunks", "f32-one-head"])
 def test_decode_host_matches_device_decode(name):
-    """sikv_decode_host (query and output in host memory: page-locked, read
-    and written in place, or pageable, staged) and its prepared form give
-    exactly what sikv_decode gives on device buffers."""
+    """sikv_decode_host (query and output in host memory: page-locked, the
+    query copied in by a kernel (staged when unaligned) and the output
+    written in place; pageable, staged) and its prepared form give exactly
+    what sikv_decode gives on device buffers."""
     dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1))
     dw.encode()
     c, p = dw.cache, dw.p
@@ -141,6 +142,18 @@ def test_decode_host_matches_device_decode(name):
         sk.sikv_decode_host(p, qp, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, op, workspace=ws)
         torch.cuda.synchronize()
         assert torch.equal(op, out_d.cpu()), (name, step)
+        # page-locked but not 16-byte aligned (one element into the buffer):
+        # the query takes the staged-copy path, the output is written in place
+        n_el = qh.numel()
+        qa = torch.empty(n_el + 1, dtype=qh.dtype).pin_memory()
+        oa = torch.full((n_el + 1,), 7.0, dtype=qh.dtype).pin_memory()
+        qu, ou = qa[1:].view(qh.shape), oa[1:].view(qh.shape)
+        qu.copy_(qh)
+        assert qu.is_pinned() and ou.is_pinned() and qu.data_ptr() % 16 and ou.data_ptr() % 16
+        sk.sikv_decode_host(p, qu, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, ou, workspace=ws)
+        torch.cuda.synchronize()
+        assert ws.check() == 0
+        assert torch.equal(ou, out_d.cpu()), (name, step)
         plan = sk.DecodeHostPlan(p, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k)
         oh2 = torch.zeros_like(oh).pin_memory()
         plan(qh, oh2)
