@@ -43,10 +43,10 @@ constexpr size_t kEncSmem = kClusters * kEncThreads * 16 + kClusters / 2 * kEncT
 // at most 2^9 such values is below 2^26 in magnitude, so every partial sum is
 // an integer multiple of 2^-27 below 2^53 * 2^-27: plain fp64 additions of
 // them are exact.  Each lane adds its fast accumulators into its
-// double-double slots after at most 264 values.  A load (two rows of a warp) in which any
-// lane sees a value outside the window (zero, subnormal, tiny, huge, inf or
-// nan) is added by two-sums into the lane's double-double accumulator
-// instead.  The result is the exact sum either way.
+// double-double slots after at most 264 values.  A load (two rows of a warp)
+// in which any lane sees a value outside the window (zero, subnormal, tiny,
+// huge, inf or nan) is added by two-sums into the lane's double-double
+// accumulator instead.  The result is the exact sum either way.
 // ---------------------------------------------------------------------------
 
 // Window edges as 15-bit bf16 magnitudes (exponent and mantissa fields):
@@ -419,7 +419,7 @@ enc_mean_final(const double2 *__restrict__ part, const int32_t *__restrict__ seq
 // Channel sums of chunk blockIdx.x of segment blockIdx.y (rows past the
 // sinks only).
 template <int DT>
-__global__ void __launch_bounds__(kEncThreads, 3)
+__global__ void __launch_bounds__(kEncThreads, kEncCtasPerSm)
 enc_mean_partial(const void *__restrict__ K, const int32_t *__restrict__ seq_lens, int hkv, int nmax,
                  int num_sinks, int chunk, int nchunks, double2 *__restrict__ part, int32_t *status) {
     constexpr int EB = ElemBytes<DT>::value;
@@ -438,7 +438,7 @@ enc_mean_partial(const void *__restrict__ K, const int32_t *__restrict__ seq_len
 
 // Codes and cluster partials of chunk blockIdx.x of segment blockIdx.y.
 template <int DT>
-__global__ void __launch_bounds__(kEncThreads, 3)
+__global__ void __launch_bounds__(kEncThreads, kEncCtasPerSm)
 enc_codes_partial(const void *__restrict__ K, const int32_t *__restrict__ seq_lens, const float *__restrict__ mu,
                   int hkv, int nmax, int num_sinks, int chunk, int nchunks, uint8_t *__restrict__ codes,
                   double *__restrict__ cb_part, int32_t *__restrict__ cnt_part, int32_t *status) {
