@@ -287,15 +287,18 @@ topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_le
 // Cluster top-k.  Segment s is cut into C chunks of `chunk` scores, one CTA
 // of 512 threads per chunk, the C CTAs forming one thread-block cluster.
 // Each CTA keeps its chunk's order-preserving keys in shared memory.  The k-th
-// largest key T is found digit by digit (bits 31-20, 19-8, 7-0): every CTA
-// histograms the digit of its keys that match the digits found so far and
-// adds the counts at or above its own need-th largest into the leader's
-// histogram (distributed shared memory); the leader finds the digit where the
-// running count from the top reaches the number still needed and hands it to
-// every CTA.  Then every CTA
-// counts its keys above T and equal to T, reads the other CTAs' counts, and
-// writes its selected tokens in ascending token order at its place: the
-// ties (keys equal to T) are taken lowest token first.
+// largest key T is found digit by digit: every CTA histograms the top 12 bits
+// of its keys and adds the counts at or above its own need-th largest into
+// the leader's histogram (distributed shared memory); the leader finds the
+// digit where the running count from the top reaches k and hands every CTA
+// the digit, the count above it and how many keys share it.  When at most
+// kKCandCap keys share it, every CTA copies its keys of that digit into the
+// leader, which finds T among them alone (bits 19-10, then 9-0).  Otherwise
+// two more cluster-wide levels follow (bits 19-8, then 7-0).  Then every CTA
+// counts its keys above T and equal to T (one ballot pass that also keeps
+// per-group masks), reads the other CTAs' counts, and writes its selected
+// tokens in ascending token order at its place from the masks: the ties
+// (keys equal to T) are taken lowest token first.
 // ---------------------------------------------------------------------------
 
 constexpr int kKT = 512;                  // threads per CTA (two CTAs per SM at 64 registers)
@@ -372,7 +375,8 @@ topk_cluster_kernel(const float *__restrict__ scores, const int32_t *__restrict_
     cluster_arrive_cta();                                    // the leader's histogram is zero
     const uint32_t mh_leader = dsmem_map(&sh.mhist[0], 0);
 
-    // the k-th key, digit by digit (bits 31-20, 19-8, 7-0)
+    // the k-th key, digit by digit (bits 31-20, then 19-8 and 7-0 unless the
+    // leader finishes from the first digit's keys)
     uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
     bool fast = false;
 #pragma unroll 1
