@@ -6,7 +6,8 @@
 //
 // Two kernels.  The cluster kernel (below) splits each segment's scores over
 // a thread-block cluster; the single-CTA kernel (one CTA of 1024 threads per
-// segment) serves segments longer than a cluster holds:
+// segment) serves segments longer than a cluster holds and shapes whose
+// cluster would hold one CTA:
 //   1. min / max of the scores;
 //   2. 4096-bin histogram linear in the score over [min, max] (a monotone
 //      map, so every token in a higher bin has a strictly higher score);
