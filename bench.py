@@ -653,10 +653,11 @@ def run_sikv(args):
     })
     del km_codes, km_cb, km_cnt, ws_km
 
-    # end to end through the public API: every step is one sikv_decode_host
-    # call (a prepared DecodeHostPlan per cache replica) on that step's query
-    # and output in page-locked host memory, which the kernels read and write
-    # over the host link; no graph
+    # end to end through the public API: every step is one
+    # sikv_decode_host_plan_run call (a DecodeHostPlan per cache replica,
+    # created before the timed region) on that step's query and output in
+    # page-locked host memory; each call copies the query in over the host
+    # link, decodes, and copies the output back
     e2e = None
     if not args.no_e2e:
         qh = torch.from_numpy(qs_host.view(np.int16) if w.dtype == "bf16" else qs_host)
@@ -683,8 +684,9 @@ def run_sikv(args):
         e2e = {"value": world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(qh[0].numel() * qh.element_size()),
                "d2h_bytes_per_step": int(oh[0].numel() * oh.element_size()),
-               "api": "sikv_decode_host (C ABI) on page-locked host buffers, one call per step; the "
-                      "kernels read the query and write the output over the host link"}
+               "api": "sikv_decode_host_plan_run (C ABI) on page-locked host buffers, one call per step: "
+                      "a graph captured at plan creation (query copy kernel, decode, output copy kernel) "
+                      "re-pointed at the step's buffers and launched"}
 
     # prefill encoder at the extreme-context shape (B=1, 32/8 heads, 512K keys
     # per head, the same generator with drift): keys encoded per second over

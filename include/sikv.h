@@ -287,6 +287,41 @@ SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, 
                                       void *workspace, size_t workspace_bytes, sikv_stream_t stream);
 
 /*
+ * sikv_decode_host_plan -- sikv_decode_host for a serving loop that decodes
+ * the same cache step after step: create() captures once, on the current
+ * device, a CUDA graph of the step (a kernel that copies the query from
+ * page-locked host memory into the workspace, the decode kernels, a kernel
+ * that copies the output to page-locked host memory); run() points the two
+ * copies at this step's buffers and launches the graph on `stream`, which
+ * removes the gaps between separately launched kernels.  Same result bytes
+ * as sikv_decode_host.
+ *  - create: arguments as for sikv_decode_host (all device pointers and the
+ *    workspace, sikv_decode_host_workspace_size() bytes, zeroed once by
+ *    sikv_workspace_init, which the plan then owns for its lifetime: do not
+ *    use it for other calls).  *plan receives the handle.  Returns the
+ *    argument errors of sikv_decode_host, SIKV_ERR_INVALID_ARG for a null
+ *    plan pointer, SIKV_ERR_CUDA when the capture fails.
+ *  - run: q_host and out_host are [B][Hq][D] in the cache dtype.  Page-locked
+ *    buffers aligned to 16 bytes take the graph; others take
+ *    sikv_decode_host's staged path on the same workspace.  Returns once
+ *    enqueued; out_host is valid after `stream` is synchronized.  Calls on
+ *    one plan must not overlap on the device (they share the workspace);
+ *    a plan is not thread-safe.
+ *  - destroy: frees the graph (the workspace stays the caller's); NULL is a
+ *    no-op.  Call it after the plan's work has finished.
+ * The paper has no counterpart: this is the host-facing form of the decode
+ * step [SIKV 2.1.2-2.1.4].
+ */
+typedef struct sikv_host_plan sikv_host_plan;
+SIKV_API sikv_status sikv_decode_host_plan_create(const sikv_params *p, const void *K, const void *V,
+                                                  const uint8_t *codes, const float *codebook, const float *mu,
+                                                  const int32_t *seq_lens, const int32_t *k_per_seq, void *workspace,
+                                                  size_t workspace_bytes, sikv_host_plan **plan);
+SIKV_API sikv_status sikv_decode_host_plan_run(sikv_host_plan *plan, const void *q_host, void *out_host,
+                                               sikv_stream_t stream);
+SIKV_API void sikv_decode_host_plan_destroy(sikv_host_plan *plan);
+
+/*
  * Comparison baselines -- not the method.  The pages compare the compressed-
  * domain retrieval with full dot-product scoring [SIKV 2.1.2] and the sparse
  * attention with dense attention [SIKV 2.1.4], and quote the speed-ups of

@@ -44,7 +44,8 @@ EXPORTED = ("sikv_version", "sikv_status_string", "sikv_workspace_init", "sikv_c
             "sikv_sparse_attn_static", "sikv_decode_host_workspace_size", "sikv_decode_host",
             "sikv_append_workspace_size", "sikv_append_codes", "sikv_dense_attn_workspace_size",
             "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_workspace_size", "sikv_kmeans_codebook",
-            "sikv_quantize_values_workspace_size", "sikv_quantize_values", "sikv_decode_qv", "sikv_sparse_attn_qv")
+            "sikv_quantize_values_workspace_size", "sikv_quantize_values", "sikv_decode_qv", "sikv_sparse_attn_qv",
+            "sikv_decode_host_plan_create", "sikv_decode_host_plan_run", "sikv_decode_host_plan_destroy")
 
 VQ_ROW_BYTES = 48     # a token's 2-bit value row: 32 bytes of levels + 4 (min, step) fp16 pairs
 
@@ -125,6 +126,10 @@ def lib() -> ctypes.CDLL:
         L.sikv_sparse_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_decode_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sikv_decode_host_plan_create.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(vp)]
+        L.sikv_decode_host_plan_run.argtypes = [vp, vp, vp, vp]
+        L.sikv_decode_host_plan_destroy.argtypes = [vp]
+        L.sikv_decode_host_plan_destroy.restype = None
         L.sikv_append_codes.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_dense_score.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         L.sikv_dense_attn.argtypes = [pp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -135,7 +140,8 @@ def lib() -> ctypes.CDLL:
         for n in ("sikv_workspace_init", "sikv_check_device_status", "sikv_encode_keys", "sikv_score",
                   "sikv_topk", "sikv_sparse_attn", "sikv_decode", "sikv_decode_host", "sikv_append_codes",
                   "sikv_dense_score", "sikv_dense_attn", "sikv_kmeans_codebook", "sikv_quantize_values",
-                  "sikv_decode_qv", "sikv_sparse_attn_qv"):
+                  "sikv_decode_qv", "sikv_sparse_attn_qv", "sikv_decode_host_plan_create",
+                  "sikv_decode_host_plan_run"):
             getattr(L, n).restype = st
         _LIB = L
     return _LIB
@@ -426,12 +432,16 @@ def sikv_decode_host(p: Params, q_host, K, V, codes, codebook, mu, seq_lens, k_p
 
 
 class DecodeHostPlan:
-    """sikv_decode_host with the device-side arguments checked once.
+    """A host-facing decode step prepared once for one cache
+    (sikv_decode_host_plan_*).
 
     A serving loop that keeps queries and outputs on the host builds one plan
-    per cache and calls it once per step with the step's host buffers (pinned
-    CPU tensors of shape [B][Hq][D] and the cache's dtype); each call is one
-    C call that enqueues the upload, the decode step and the download.
+    per cache and calls it once per step with the step's host buffers (CPU
+    tensors of shape [B][Hq][D] and the cache's dtype).  Construction captures
+    the step as a CUDA graph on the plan's own workspace; each call points its
+    query and output copies at the given buffers and launches it on the
+    plan's stream (page-locked buffers aligned to 16 bytes; others take
+    sikv_decode_host's staged path).  Synchronize before reading the output.
     """
 
     def __init__(self, p: Params, K, V, codes, codebook, mu, seq_lens, k_per_seq, workspace=None, stream=None):
@@ -442,8 +452,15 @@ class DecodeHostPlan:
         self._shape = (p.batch, p.num_q_heads, p.head_dim)
         self._dtype = p.torch_dtype
         self._stream = _stream(stream, dev)
-        self._pref = ctypes.byref(p)
-        self._fn = lib().sikv_decode_host
+        L = lib()
+        self._destroy = L.sikv_decode_host_plan_destroy
+        self._run = L.sikv_decode_host_plan_run
+        # the workspace was zeroed on the plan's stream, where every replay runs
+        handle = ctypes.c_void_p()
+        _check(L.sikv_decode_host_plan_create(ctypes.byref(p), *self._dargs, self.workspace.ptr,
+                                              self.workspace.nbytes, ctypes.byref(handle)),
+               "sikv_decode_host_plan_create")
+        self._plan = handle
 
     def __call__(self, q_host, out_host):
         if q_host.is_cuda or out_host.is_cuda or q_host.dtype != self._dtype or out_host.dtype != self._dtype \
@@ -451,10 +468,21 @@ class DecodeHostPlan:
                 or not (q_host.is_contiguous() and out_host.is_contiguous()):
             _host_ptr(q_host, "q_host", self._dtype, self._shape)       # raises with the reason
             _host_ptr(out_host, "out_host", self._dtype, self._shape)
-        st = self._fn(self._pref, q_host.data_ptr(), *self._dargs, out_host.data_ptr(), self.workspace.ptr,
-                      self.workspace.nbytes, self._stream)
+        st = self._run(self._plan, q_host.data_ptr(), out_host.data_ptr(), self._stream)
         if st != 0:
-            raise SikvError(st, "sikv_decode_host")
+            raise SikvError(st, "sikv_decode_host_plan_run")
+
+    def close(self):
+        """Free the plan's graph (after its work has finished)."""
+        if getattr(self, "_plan", None) is not None and self._plan.value:
+            self._destroy(self._plan)
+        self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ----------------------------------------------------------------------------

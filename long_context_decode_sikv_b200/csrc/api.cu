@@ -4,10 +4,32 @@
 #include <atomic>
 #include <string.h>
 
+#include <new>
+#include <vector>
+
 #include "sikv_common.cuh"
 #include "sikv_internal.h"
 
 using namespace sikv;
+
+// A captured host-facing decode step (sikv_decode_host_plan_*): the graph
+// [query copy -> decode kernels -> output copy] on the plan's workspace, and
+// the two copy nodes that each run re-points.
+struct sikv_host_plan {
+    sikv_params p;
+    const void *K, *V;
+    const uint8_t *codes;
+    const float *codebook, *mu;
+    const int32_t *seq_lens, *k_per_seq;
+    char *ws;
+    size_t ws_bytes;
+    uint4 *q_slot, *out_slot;           // the workspace's device copies of q and of the output
+    int n16;                            // 16-byte words of one q (= one output) tensor
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    cudaGraphNode_t up, down;
+    cudaKernelNodeParams up_kp, down_kp;
+};
 
 namespace {
 
@@ -128,14 +150,16 @@ HostLayout host_layout(const sikv_params &p, size_t decode_total) {
     return H;
 }
 
-// The device address of a page-locked host buffer, or null for pageable
-// memory (which then goes through a staged copy).
-// Copies n16 16-byte words from host-mapped memory into device memory: each
-// word crosses the host link once, and a warp reads 512 contiguous bytes.
-__global__ void __launch_bounds__(256) upload16_kernel(const uint4 *src, uint4 *__restrict__ dst, int n16) {
+// Copies n16 16-byte words between host-mapped and device memory: each word
+// crosses the host link once, and a warp moves 512 contiguous bytes.
+__global__ void __launch_bounds__(256) copy16_kernel(const uint4 *src, uint4 *dst, int n16) {
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += gridDim.x * blockDim.x) dst[i] = src[i];
 }
 
+int copy16_grid(int n16) { return std::min((n16 + 255) / 256, 64); }
+
+// The device address of a page-locked host buffer, or null for pageable
+// memory (which then goes through a staged copy).
 void *device_view(const void *host) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
@@ -536,8 +560,8 @@ sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const voi
     char *q_dev = ws + H.q;
     if (q_view && (reinterpret_cast<uintptr_t>(q_view) & 15u) == 0 && H.bytes % 16 == 0) {
         const int n16 = static_cast<int>(H.bytes / 16);
-        sikv::upload16_kernel<<<std::min((n16 + 255) / 256, 64), 256, 0, s>>>(
-            static_cast<const uint4 *>(q_view), reinterpret_cast<uint4 *>(q_dev), n16);
+        sikv::copy16_kernel<<<sikv::copy16_grid(n16), 256, 0, s>>>(static_cast<const uint4 *>(q_view),
+                                                                   reinterpret_cast<uint4 *>(q_dev), n16);
         if (cudaGetLastError() != cudaSuccess) return SIKV_ERR_CUDA;
     } else if (cudaMemcpyAsync(q_dev, q_host, H.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
         return SIKV_ERR_CUDA;
@@ -547,6 +571,137 @@ sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, const voi
     if (!out_dev &&
         cudaMemcpyAsync(out_host, ws + H.out, H.bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return SIKV_ERR_CUDA;
+    return SIKV_OK;
+}
+
+void sikv_decode_host_plan_destroy(sikv_host_plan *plan) {
+    if (!plan) return;
+    if (plan->exec) cudaGraphExecDestroy(plan->exec);
+    if (plan->graph) cudaGraphDestroy(plan->graph);
+    delete plan;
+}
+
+sikv_status sikv_decode_host_plan_create(const sikv_params *p, const void *K, const void *V, const uint8_t *codes,
+                                         const float *codebook, const float *mu, const int32_t *seq_lens,
+                                         const int32_t *k_per_seq, void *workspace, size_t workspace_bytes,
+                                         sikv_host_plan **plan) {
+    if (!plan) return SIKV_ERR_INVALID_ARG;
+    *plan = nullptr;
+    SIKV_TRY(check_params(p));
+    SIKV_REQUIRE_PTR(K);
+    SIKV_REQUIRE_PTR(V);
+    SIKV_REQUIRE_PTR(codes);
+    SIKV_REQUIRE_PTR(codebook);
+    SIKV_REQUIRE_PTR(mu);
+    SIKV_REQUIRE_PTR4(seq_lens);
+    SIKV_REQUIRE_PTR4(k_per_seq);
+    const size_t decode_total = decode_layout(*p).total;
+    const sikv::HostLayout H = sikv::host_layout(*p, decode_total);
+    SIKV_TRY(check_ws(workspace, workspace_bytes, H.total));
+    if (H.bytes % 16 != 0) return SIKV_ERR_UNSUPPORTED;
+    // the launch facts the decode kernels need are computed now, outside the capture
+    if (resolve_decode_path(*p, false) == 0) return SIKV_ERR_UNSUPPORTED;
+
+    sikv_host_plan *pl = new (std::nothrow) sikv_host_plan();
+    if (!pl) return SIKV_ERR_CUDA;
+    pl->p = *p;
+    pl->K = K;
+    pl->V = V;
+    pl->codes = codes;
+    pl->codebook = codebook;
+    pl->mu = mu;
+    pl->seq_lens = seq_lens;
+    pl->k_per_seq = k_per_seq;
+    pl->ws = static_cast<char *>(workspace);
+    pl->ws_bytes = workspace_bytes;
+    pl->q_slot = reinterpret_cast<uint4 *>(pl->ws + H.q);
+    pl->out_slot = reinterpret_cast<uint4 *>(pl->ws + H.out);
+    pl->n16 = static_cast<int>(H.bytes / 16);
+
+    // capture on a private stream: nothing runs now.  The copies are captured
+    // with placeholder host ends (the workspace slots themselves) that every
+    // run replaces.
+    cudaStream_t cs = nullptr;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) {
+        delete pl;
+        return SIKV_ERR_CUDA;
+    }
+    sikv_status st = SIKV_OK;
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        st = SIKV_ERR_CUDA;
+    } else {
+        const int g = sikv::copy16_grid(pl->n16);
+        sikv::copy16_kernel<<<g, 256, 0, cs>>>(pl->q_slot, pl->q_slot, pl->n16);
+        st = sikv::decode_step(*p, pl->q_slot, K, V, nullptr, codes, codebook, mu, seq_lens, k_per_seq, pl->out_slot,
+                               nullptr, nullptr, workspace, decode_total, cs);
+        sikv::copy16_kernel<<<g, 256, 0, cs>>>(pl->out_slot, pl->out_slot, pl->n16);
+        cudaGraph_t graph = nullptr;
+        const cudaError_t e = cudaStreamEndCapture(cs, &graph);      // always ends the capture
+        pl->graph = graph;
+        if (st == SIKV_OK && (e != cudaSuccess || !graph)) st = SIKV_ERR_CUDA;
+    }
+    cudaStreamDestroy(cs);
+    cudaGetLastError();
+    // the two copy nodes: the one writing the q slot and the one reading the output slot
+    if (st == SIKV_OK) {
+        size_t n = 0;
+        if (cudaGraphGetNodes(pl->graph, nullptr, &n) != cudaSuccess) st = SIKV_ERR_CUDA;
+        std::vector<cudaGraphNode_t> nodes(n);
+        if (st == SIKV_OK && n && cudaGraphGetNodes(pl->graph, nodes.data(), &n) != cudaSuccess) st = SIKV_ERR_CUDA;
+        for (size_t i = 0; st == SIKV_OK && i < n; ++i) {
+            cudaGraphNodeType type;
+            if (cudaGraphNodeGetType(nodes[i], &type) != cudaSuccess || type != cudaGraphNodeTypeKernel) continue;
+            cudaKernelNodeParams kp;
+            if (cudaGraphKernelNodeGetParams(nodes[i], &kp) != cudaSuccess) continue;
+            if (kp.func != reinterpret_cast<void *>(sikv::copy16_kernel) || !kp.kernelParams) continue;
+            const uint4 *src = *static_cast<const uint4 *const *>(kp.kernelParams[0]);
+            uint4 *dst = *static_cast<uint4 *const *>(kp.kernelParams[1]);
+            if (dst == pl->q_slot && src == pl->q_slot) {
+                pl->up = nodes[i];
+                pl->up_kp = kp;
+            } else if (src == pl->out_slot) {
+                pl->down = nodes[i];
+                pl->down_kp = kp;
+            }
+        }
+        if (st == SIKV_OK && (!pl->up || !pl->down)) st = SIKV_ERR_CUDA;
+    }
+    if (st == SIKV_OK && cudaGraphInstantiate(&pl->exec, pl->graph, 0) != cudaSuccess) st = SIKV_ERR_CUDA;
+    cudaGetLastError();
+    if (st != SIKV_OK) {
+        sikv_decode_host_plan_destroy(pl);
+        return st;
+    }
+    *plan = pl;
+    return SIKV_OK;
+}
+
+sikv_status sikv_decode_host_plan_run(sikv_host_plan *plan, const void *q_host, void *out_host,
+                                      sikv_stream_t stream) {
+    if (!plan || !q_host || !out_host) return SIKV_ERR_INVALID_ARG;
+    const void *qv = sikv::device_view(q_host);
+    void *ov = sikv::device_view(out_host);
+    const bool graphed = qv && ov && (reinterpret_cast<uintptr_t>(qv) & 15u) == 0 &&
+                         (reinterpret_cast<uintptr_t>(ov) & 15u) == 0;
+    if (!graphed)
+        return sikv_decode_host(&plan->p, q_host, plan->K, plan->V, plan->codes, plan->codebook, plan->mu,
+                                plan->seq_lens, plan->k_per_seq, out_host, plan->ws, plan->ws_bytes, stream);
+    int n16 = plan->n16;
+    const uint4 *up_src = static_cast<const uint4 *>(qv);
+    uint4 *up_dst = plan->q_slot;
+    void *up_args[] = {&up_src, &up_dst, &n16};
+    cudaKernelNodeParams kp = plan->up_kp;
+    kp.kernelParams = up_args;
+    kp.extra = nullptr;
+    if (cudaGraphExecKernelNodeSetParams(plan->exec, plan->up, &kp) != cudaSuccess) return SIKV_ERR_CUDA;
+    const uint4 *down_src = plan->out_slot;
+    uint4 *down_dst = static_cast<uint4 *>(ov);
+    void *down_args[] = {&down_src, &down_dst, &n16};
+    kp = plan->down_kp;
+    kp.kernelParams = down_args;
+    kp.extra = nullptr;
+    if (cudaGraphExecKernelNodeSetParams(plan->exec, plan->down, &kp) != cudaSuccess) return SIKV_ERR_CUDA;
+    if (cudaGraphLaunch(plan->exec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SIKV_ERR_CUDA;
     return SIKV_OK;
 }
 

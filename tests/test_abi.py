@@ -125,6 +125,32 @@ def test_decode_host_validates_without_launch():
     assert st == 1                                       # invalid parameters
 
 
+def test_decode_host_plan_validates_without_capture():
+    """sikv_decode_host_plan_create refuses bad arguments before any CUDA
+    call (a null handle pointer, invalid parameters, null or misaligned
+    device pointers, a missing or short workspace); run refuses a null plan
+    or null host buffers; destroy accepts NULL."""
+    p = _p()
+    L = sk.lib()
+    n_host = L.sikv_decode_host_workspace_size(ctypes.byref(p))
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    h = ctypes.c_void_p()
+    args = [fake] * 7
+    assert L.sikv_decode_host_plan_create(ctypes.byref(p), *args, ws, n_host, None) == 1
+    bad = sk.make_params("bf16", 2, 7, 2, 4096, 64, 256)
+    assert L.sikv_decode_host_plan_create(ctypes.byref(bad), *args, ws, n_host, ctypes.byref(h)) == 1
+    assert not h.value
+    assert L.sikv_decode_host_plan_create(ctypes.byref(p), None, *args[1:], ws, n_host, ctypes.byref(h)) == 1
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert L.sikv_decode_host_plan_create(ctypes.byref(p), odd, *args[1:], ws, n_host, ctypes.byref(h)) == 2
+    assert L.sikv_decode_host_plan_create(ctypes.byref(p), *args, None, n_host, ctypes.byref(h)) == 3
+    assert L.sikv_decode_host_plan_create(ctypes.byref(p), *args, ws, n_host - 256, ctypes.byref(h)) == 3
+    assert not h.value
+    assert L.sikv_decode_host_plan_run(None, fake, fake, None) == 1
+    L.sikv_decode_host_plan_destroy(None)
+
+
 def test_decode_host_binding_refuses_device_or_misshapen_buffers():
     p = _p()
     import torch

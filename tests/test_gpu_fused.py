@@ -121,11 +121,14 @@ def test_fused_all_scores_tied_takes_lowest_indices(path):
 def test_decode_host_matches_device_decode(name):
     """sikv_decode_host (query and output in host memory: page-locked, the
     query copied in by a kernel (staged when unaligned) and the output
-    written in place; pageable, staged) and its prepared form give exactly
-    what sikv_decode gives on device buffers."""
+    written in place; pageable, staged) and its plan (a captured graph whose
+    copies each call points at its buffers) give exactly what sikv_decode
+    gives on device buffers."""
     dw = gu.DeviceWorkload(SHAPES[name](), steps=(0, 1))
     dw.encode()
     c, p = dw.cache, dw.p
+    # one plan (a captured graph) for both steps: each call re-points its copies
+    plan = sk.DecodeHostPlan(p, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k)
     for step in (0, 1):
         out_d = torch.empty_like(dw.q[step])
         sk.sikv_decode(p, dw.q[step], c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k, out_d).check()
@@ -154,13 +157,20 @@ def test_decode_host_matches_device_decode(name):
         torch.cuda.synchronize()
         assert ws.check() == 0
         assert torch.equal(ou, out_d.cpu()), (name, step)
-        plan = sk.DecodeHostPlan(p, c.K, c.V, c.codes, c.codebook, c.mu, dw.seq_lens, dw.k)
         oh2 = torch.zeros_like(oh).pin_memory()
         plan(qh, oh2)
         plan(qh, oh2)                                   # repeated calls: same answer
         torch.cuda.synchronize()
         assert plan.workspace.check() == 0
         assert torch.equal(oh2, out_d.cpu()), (name, step)
+        # buffers the graph does not take (unaligned, pageable): the staged path
+        ou.fill_(7.0)
+        plan(qu, ou)
+        op.fill_(7.0)
+        plan(qp, op)
+        torch.cuda.synchronize()
+        assert torch.equal(ou, out_d.cpu()) and torch.equal(op, out_d.cpu()), (name, step)
+    plan.close()
 
 
 @pytest.mark.parametrize("path", sorted(PATHS))
