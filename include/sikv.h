@@ -297,16 +297,16 @@ SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, 
  * as sikv_decode_host.
  *  - create: arguments as for sikv_decode_host (all device pointers and the
  *    workspace, sikv_decode_host_workspace_size() bytes, zeroed once by
- *    sikv_workspace_init, which the plan then owns for its lifetime: do not
- *    use it for other calls).  *plan receives the handle.  Returns the
+ *    sikv_workspace_init; the plan keeps using it, so calls that share it --
+ *    this plan's runs, other plans, other entry points -- must not overlap
+ *    on the device).  *plan receives the handle.  Returns the
  *    argument errors of sikv_decode_host, SIKV_ERR_INVALID_ARG for a null
  *    plan pointer, SIKV_ERR_CUDA when the capture fails.
  *  - run: q_host and out_host are [B][Hq][D] in the cache dtype.  Page-locked
  *    buffers aligned to 16 bytes take the graph; others take
  *    sikv_decode_host's staged path on the same workspace.  Returns once
- *    enqueued; out_host is valid after `stream` is synchronized.  Calls on
- *    one plan must not overlap on the device (they share the workspace);
- *    a plan is not thread-safe.
+ *    enqueued; out_host is valid after `stream` is synchronized.  A plan is
+ *    not thread-safe.
  *  - destroy: frees the graph (the workspace stays the caller's); NULL is a
  *    no-op.  Call it after the plan's work has finished.
  * The paper has no counterpart: this is the host-facing form of the decode
