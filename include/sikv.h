@@ -309,6 +309,9 @@ SIKV_API sikv_status sikv_decode_host(const sikv_params *p, const void *q_host, 
  *    not thread-safe.
  *  - destroy: frees the graph (the workspace stays the caller's); NULL is a
  *    no-op.  Call it after the plan's work has finished.
+ * The plan is a caller-owned host object; the executable graph's resources
+ * are the CUDA runtime's, held from create to destroy (the library itself
+ * still allocates no device memory).
  * The paper has no counterpart: this is the host-facing form of the decode
  * step [SIKV 2.1.2-2.1.4].
  */
